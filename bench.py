@@ -1,0 +1,496 @@
+"""Benchmark of the verification sampler (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config batched|single|greedy|tree|tree-stochastic]
+
+A step is one verification call over one batch of synthetic inputs: for the
+default workload, 64 requests x 8 drafts over a 128256-entry bf16
+vocabulary at T = 0.7 (576 target rows + 512 draft rows = 279.09 MB of
+logits).  The metric is verify rows per second (target rows of the batch
+per second), whole job; achieved HBM GB/s is reported in `roofline`.
+
+N > 1 (launched by torchrun, one process per GPU): every rank verifies its
+own batch (requests are independent: no collective on the data path); the
+time is the max over ranks of the device-timed region.
+
+`--impl reference` times the fp64 CPU oracle on the host, on a bounded
+sample of the same workload (rank 0 only).
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "verify rows/s and achieved HBM GB/s (B=64, k=8, V=128256 bf16, 1 B200)"
+L2_BYTES = 126 * 2 ** 20
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------- workloads
+def make_workload(name, seed):
+    from speculative_decoding_verification_87_b200 import workloads as wl
+    if name == "batched":
+        return wl.config_batched(seed=seed)
+    if name == "single":
+        return wl.config_single(seed=seed)
+    if name == "greedy":
+        return wl.config_greedy(seed=seed)
+    if name in ("tree", "tree-stochastic"):
+        return wl.config_tree(seed=seed)
+    raise ValueError(name)
+
+
+def workload_facts(name, w):
+    """(rows per step, algorithmic bytes per step, config dict)."""
+    esz = 2 if w.dtype == "bf16" else 4
+    if name in ("batched", "single"):
+        B, k, V = w.batch, w.k, w.vocab
+        rows = B * (k + 1)
+        logits = (B * (k + 1) + B * k) * V * esz
+        io = B * k * 4 + B * (k + 1) * 4 + B * 4
+        cfg = dict(workload=f"linear stochastic verify B={B} k={k} V={V} {w.dtype} T={w.temperature}",
+                   batch=B, k=k, vocab=V, temperature=w.temperature)
+    elif name == "greedy":
+        B, k, V = w.batch, w.k, w.vocab
+        rows = B * (k + 1)
+        logits = B * (k + 1) * V * esz
+        io = B * k * 4 + B * (k + 1) * 4 + B * 4
+        cfg = dict(workload=f"linear greedy verify B={B} k={k} V={V} {w.dtype}", batch=B, k=k,
+                   vocab=V)
+    else:
+        B, N, V = w.batch, w.num_nodes, w.vocab
+        rows = B * N
+        stoch = name == "tree-stochastic"
+        nonleaf = sum(int(len(set(w.parents[b, 1:].tolist()))) for b in range(B))
+        logits = (B * N + (nonleaf if stoch else 0)) * V * esz
+        io = 2 * B * N * 4 + 2 * B * (w.max_depth + 1) * 4 + B * 4
+        cfg = dict(workload=f"tree {'stochastic' if stoch else 'greedy'} verify B={B} N={N} "
+                            f"depth={w.max_depth} V={V} {w.dtype}", batch=B, nodes=N, vocab=V)
+    return rows, logits + io, cfg
+
+
+# ------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    def __init__(self, index, period=0.01):
+        self.index, self.period = index, period
+        self.samples = []
+        self._stop = threading.Event()
+        self._thr = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+            self._sample()
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        except Exception:
+            self.ok = False
+        return self
+
+    def _sample(self):
+        nv = self._nv
+        sm = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+        reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        self.samples.append((sm, reasons))
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                break
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thr is not None:
+            self._thr.join()
+        if self.ok:
+            try:
+                self._sample()
+            except Exception:
+                pass
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        nv = self._nv
+        names = {
+            "gpu_idle": getattr(nv, "nvmlClocksEventReasonGpuIdle", 0x1),
+            "applications_clocks_setting": getattr(nv, "nvmlClocksEventReasonApplicationsClocksSetting", 0x2),
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "sync_boost": getattr(nv, "nvmlClocksEventReasonSyncBoost", 0x10),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "hw_power_brake_slowdown": getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        seen = 0
+        for _, r in self.samples:
+            seen |= r
+        reasons = [n for n, bit in names.items() if seen & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(s for s, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------- distributed
+def dist_setup(n_gpus):
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def max_over_ranks(value, world, device):
+    """Max of a float over all ranks (identity at world size 1)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# -------------------------------------------------------------- our arm
+class Runner:
+    """Binds one workload's device buffers to the C-ABI call of its mode."""
+
+    def __init__(self, name, w, device):
+        import torch
+        from speculative_decoding_verification_87_b200 import binding
+        self.binding, self.name, self.w, self.device = binding, name, w, device
+
+        def dev(a):
+            t = torch.from_numpy(np.ascontiguousarray(a))
+            if a.dtype == np.uint16:
+                t = t.view(torch.bfloat16)
+            return t.to(device)
+
+        self.dev = dev
+        self.target = dev(w.target)
+        self.draft = dev(w.draft)
+        if name in ("tree", "tree-stochastic"):
+            self.tokens = dev(w.node_tokens)
+            self.parents = dev(w.parents)
+            W = w.max_depth + 1
+            self.out = torch.empty((w.batch, W), dtype=torch.int32, device=device)
+            self.kernels_per_call = 1 if name == "tree" else 2
+        else:
+            self.tokens = dev(w.tokens.astype(np.int32))
+            self.out = torch.empty((w.batch, w.k + 1), dtype=torch.int32, device=device)
+            self.kernels_per_call = {"greedy": 1}.get(name, 3)
+        self.acc = torch.empty((w.batch,), dtype=torch.int32, device=device)
+
+    def call(self, offset, target=None, draft=None, tokens=None):
+        b, w = self.binding, self.w
+        target = self.target if target is None else target
+        draft = self.draft if draft is None else draft
+        tokens = self.tokens if tokens is None else tokens
+        if self.name in ("batched", "single"):
+            b.spec_verify_linear(target, draft, tokens, w.vocab, w.temperature, 1234, offset,
+                                 out_tokens=self.out, accepted_len=self.acc)
+        elif self.name == "greedy":
+            b.spec_verify_greedy(target, tokens, w.vocab, out_tokens=self.out,
+                                 accepted_len=self.acc)
+        else:
+            b.spec_verify_tree(target, draft, tokens, self.parents, w.max_depth, w.vocab,
+                               self.name == "tree-stochastic", w.temperature, 1234, offset,
+                               out_tokens=self.out, accepted_len=self.acc)
+
+
+def run_ours(args, rank, world, local):
+    import torch
+    from speculative_decoding_verification_87_b200 import binding, build
+    if rank == 0:
+        build.build()
+    barrier(world)
+    binding.load_library()
+    device = torch.device("cuda", local)
+    name = args.config
+    sets = [make_workload(name, seed=1000 * rank + s) for s in range(2)]
+    rows, alg_bytes, cfg = workload_facts(name, sets[0])
+    runners = [Runner(name, w, device) for w in sets]
+    stream = torch.cuda.current_stream(device)
+
+    # warm-up
+    for i in range(args.warmup):
+        runners[i % 2].call(offset=i)
+    torch.cuda.synchronize(device)
+    barrier(world)
+
+    # device-timed region: exactly K steps, inputs alternate between two
+    # resident sets (each larger than L2)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize(device)
+        barrier(world)
+        start.record(stream)
+        for i in range(args.steps):
+            runners[i % 2].call(offset=args.warmup + i)
+        stop.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(world)
+    ms = start.elapsed_time(stop)
+    ms_max = max_over_ranks(ms, world, device)
+    value = rows * args.steps * world / (ms_max / 1e3)
+    step_s = ms_max / 1e3 / args.steps
+    peak, peak_src = _peaks()
+    achieved = alg_bytes / step_s / 1e9
+
+    # end to end through the same API from pinned host buffers: each step
+    # copies its inputs host->device, verifies, and reads the outputs back
+    e2e = run_e2e(args, runners[0], sets[0], device, world)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": value,
+            "unit": "rows/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_max / args.steps,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": sets[0].dtype,
+            "data": "synthetic",
+            "config": dict(cfg, parallelism=f"dp{world} (independent request shards)",
+                           l2="inputs larger than L2: 2 resident input sets of "
+                              f"{alg_bytes / 1e6:.1f} MB alternate",
+                           requests_per_rank=sets[0].batch),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
+                         if peak_src == "measured" else "fallback",
+                         "kernel": "whole verification call (all kernels of a step)",
+                         "algorithmic_bytes_per_launch": alg_bytes},
+            "e2e": e2e,
+            "gpu_launches": runners[0].kernels_per_call * args.steps,
+            "clocks": clk.summary(),
+            "tokens_per_s": None,
+        }
+        if args.cpu_baseline and world == 1:
+            line["cpu_baseline"] = oracle_baseline(name, sets[0], rows)
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, runner, w, device, world):
+    import torch
+    tgt_h = torch.from_numpy(np.ascontiguousarray(w.target)).pin_memory()
+    drf_h = torch.from_numpy(np.ascontiguousarray(w.draft)).pin_memory()
+    tok_src = w.node_tokens if runner.name in ("tree", "tree-stochastic") else w.tokens
+    tok_h = torch.from_numpy(np.ascontiguousarray(tok_src.astype(np.int32))).pin_memory()
+    if w.target.dtype == np.uint16:
+        tgt_h, drf_h = tgt_h.view(torch.bfloat16), drf_h.view(torch.bfloat16)
+    tgt_d = torch.empty(tgt_h.shape, dtype=tgt_h.dtype, device=device)
+    drf_d = torch.empty(drf_h.shape, dtype=drf_h.dtype, device=device)
+    tok_d = torch.empty(tok_h.shape, dtype=tok_h.dtype, device=device)
+    out_h = torch.empty(runner.out.shape, dtype=torch.int32).pin_memory()
+    acc_h = torch.empty(runner.acc.shape, dtype=torch.int32).pin_memory()
+    needs_draft = runner.name not in ("greedy", "tree")
+    stream = torch.cuda.current_stream(device)
+
+    def step(i):
+        tgt_d.copy_(tgt_h, non_blocking=True)
+        if needs_draft:
+            drf_d.copy_(drf_h, non_blocking=True)
+        tok_d.copy_(tok_h, non_blocking=True)
+        runner.call(offset=i, target=tgt_d, draft=drf_d, tokens=tok_d)
+        out_h.copy_(runner.out, non_blocking=True)
+        acc_h.copy_(runner.acc, non_blocking=True)
+
+    for i in range(max(1, min(args.warmup, 3))):
+        step(i)
+    torch.cuda.synchronize(device)
+    barrier(world)
+    steps = max(1, min(args.steps, 20))
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(steps):
+        step(100 + i)
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    ms = max_over_ranks(a.elapsed_time(b), world, device)
+    rows, _, _ = workload_facts(runner.name, w)
+    h2d = tgt_h.numel() * tgt_h.element_size() + tok_h.numel() * 4
+    if needs_draft:
+        h2d += drf_h.numel() * drf_h.element_size()
+    d2h = (out_h.numel() + acc_h.numel()) * 4
+    return {"value": rows * steps * world / (ms / 1e3), "unit": "rows/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps}
+
+
+# ------------------------------------------------------------ oracle timing
+def oracle_sample(name, w, max_requests):
+    """A bounded slice of the workload (first requests) for the CPU oracle."""
+    import copy
+    s = copy.copy(w)
+    n = min(max_requests, w.batch)
+    s.target = np.ascontiguousarray(w.target[:n])
+    s.draft = np.ascontiguousarray(w.draft[:n])
+    if hasattr(w, "tokens"):
+        s.tokens = np.ascontiguousarray(w.tokens[:n])
+    if hasattr(w, "node_tokens"):
+        s.node_tokens = np.ascontiguousarray(w.node_tokens[:n])
+        s.parents = np.ascontiguousarray(w.parents[:n])
+    return s
+
+
+def oracle_call(name, s, offset):
+    import oracle
+    if name in ("batched", "single"):
+        oracle.verify_linear(s.target, s.draft, s.tokens, s.vocab, s.temperature, 1234, offset)
+        return s.target.shape[0] * s.target.shape[1]
+    if name == "greedy":
+        oracle.verify_greedy(s.target, s.tokens, s.vocab)
+        return s.target.shape[0] * s.target.shape[1]
+    oracle.verify_tree(s.target, s.draft, s.node_tokens, s.parents, s.max_depth, s.vocab,
+                       name == "tree-stochastic", s.temperature, 1234, offset)
+    return s.target.shape[0] * s.target.shape[1]
+
+
+def oracle_baseline(name, w, rows_full, budget_s=10.0, max_requests=16):
+    import oracle
+    oracle.lib()
+    s = oracle_sample(name, w, max_requests)
+    oracle_call(name, s, 0)  # warm the page cache / library
+    t0 = time.perf_counter()
+    rows = 0
+    calls = 0
+    while True:
+        rows += oracle_call(name, s, calls + 1)
+        calls += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": rows / dt, "unit": "rows/s", "cores": 1, "kind": "oracle",
+            "sample": f"{calls} oracle calls on the first {s.target.shape[0]} of {w.batch} "
+                      f"requests ({rows} target rows, {dt:.1f} s, single thread, "
+                      f"{_cpu_name()})"}
+
+
+def _cpu_name():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip() + f", nproc={os.cpu_count()}"
+    except Exception:
+        pass
+    return f"nproc={os.cpu_count()}"
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    name = args.config
+    w = make_workload(name, seed=0)
+    rows_full, alg_bytes, cfg = workload_facts(name, w)
+    import oracle
+    oracle.lib()
+    s = oracle_sample(name, w, max_requests=8)
+    for i in range(args.warmup):
+        oracle_call(name, s, i)
+    t0 = time.perf_counter()
+    rows = 0
+    for i in range(args.steps):
+        rows += oracle_call(name, s, args.warmup + i)
+    dt = time.perf_counter() - t0
+    value = rows / dt
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "rows/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": dt * 1e3 / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": dict(cfg, parallelism="host, single thread"),
+        "cpu_baseline": {"value": value, "unit": "rows/s", "cores": 1, "kind": "oracle",
+                         "sample": f"each step = one oracle call on the first "
+                                   f"{s.target.shape[0]} of {w.batch} requests "
+                                   f"({_cpu_name()})"},
+        "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="batched",
+                    choices=["batched", "single", "greedy", "tree", "tree-stochastic"])
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        run_reference(args, rank, world)
+        return
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

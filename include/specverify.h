@@ -1,0 +1,200 @@
+/*
+ * specverify.h -- C ABI of the B200 (sm_100a) speculative-decoding
+ * verification sampler, libspecverify.so.
+ *
+ * What the calls compute ("Accelerating Sonar through speculation",
+ * Perplexity 2025, section "Speculative decoding": after the draft stage come
+ * the acceptance stage and the target-generation stage; section
+ * "Target-Draft": acceptance compares the full draft and target
+ * distributions, and the target always yields one more set of logits after
+ * the accepted drafts; "Speculative decoding explained", section "Draft and
+ * verification loop": a draft is accepted outright when the target is at
+ * least as confident, otherwise with a probability that falls as the gap
+ * grows, and a rejected draft is replaced by a token drawn from an adjusted
+ * distribution, which keeps the target's output distribution exactly).
+ * The exact rule, as in Leviathan, Kalman & Matias, "Fast inference from
+ * transformers via speculative decoding": accept draft x with probability
+ * min(1, p(x)/q(x)); at the first rejection resample from
+ * norm(max(0, p - q)); if nothing is rejected, sample the bonus token from
+ * the last target row.
+ *
+ * Notation: B requests, k drafts per request, V vocabulary entries, T
+ * temperature.  p_j = softmax(target_row_j / T), q_j = softmax(draft_row_j / T).
+ *
+ * Conventions shared by every call:
+ *   - Every pointer argument is caller-owned DEVICE memory (global memory of
+ *     the current device), except where a comment says otherwise.  The
+ *     library allocates nothing, keeps no state between calls, and never
+ *     synchronises: all work is enqueued on `stream` and the outputs are
+ *     valid when the stream reaches that point.
+ *   - Logit tensors are row-major [B][rows][row_stride] of fp32 or bf16.
+ *     Only columns [0, V) of a row are read as vocabulary.  row_stride * the
+ *     element size must be a multiple of 16 bytes and every logit base
+ *     pointer 16-byte aligned (the kernels move rows in 16-byte vectors).
+ *   - Random numbers: Philox4x32-10 (Salmon et al., SC'11) with key
+ *     (seed low 32 bits, seed high 32 bits) and counter (request, position,
+ *     purpose, offset); u = (first output word >> 8) * 2^-24.  Purposes:
+ *     0 = accept test, 1 = final sample.  Equal (seed, offset) give equal
+ *     results; advance `offset` between calls for fresh randomness.
+ *   - Return value: SPEC_OK, or a negative code detected on the host before
+ *     anything is enqueued (SPEC_ECUDA: a launch failed; earlier kernels of
+ *     the same call may have run).
+ *   - Input errors the host cannot see (a token outside [0, V), a malformed
+ *     parent array, a NaN logit, a row with no finite normaliser) are
+ *     reported per request: that request's out_tokens and accepted_len are
+ *     all -1 and the matching SPEC_STATUS_* bit is OR-ed into *status when
+ *     status is non-NULL.  The kernels never trap.
+ */
+#ifndef SPECVERIFY_H
+#define SPECVERIFY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SPECVERIFY_API __attribute__((visibility("default")))
+#else
+#define SPECVERIFY_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The CUDA runtime's stream handle; repeated here so that the header needs
+ * no CUDA include.  Pass 0 for the legacy default stream. */
+typedef struct CUstream_st *cudaStream_t;
+
+typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype_t;
+
+enum {
+    SPEC_OK = 0,
+    SPEC_EINVAL = -1,        /* a size, count, temperature or NULL pointer is invalid   */
+    SPEC_EALIGN = -2,        /* a logit base or the row pitch is not 16-byte aligned    */
+    SPEC_EUNSUPPORTED = -3,  /* a size beyond the documented limits                      */
+    SPEC_ECUDA = -4,         /* a CUDA launch or query failed                            */
+    SPEC_EWORKSPACE = -5     /* workspace NULL, misaligned or smaller than required      */
+};
+
+/* Bits OR-ed into *status (device int32) by the kernels. */
+enum {
+    SPEC_STATUS_TOKEN = 1,   /* a draft or node token outside [0, V)                     */
+    SPEC_STATUS_TREE = 2,    /* parents[0] != -1, parents[i] not in [0, i), or a node
+                                deeper than max_depth                                    */
+    SPEC_STATUS_LOGIT = 4    /* a NaN logit, or a row with no finite normaliser
+                                (+inf present, or every entry -inf)                      */
+};
+
+/* Limits checked on the host. */
+#define SPEC_MAX_K 32
+#define SPEC_MAX_NODES 1024
+
+/*
+ * Bytes of device workspace a call needs for `batch` requests with
+ * `rows_per_req` logit rows each (linear: 2k+1; tree: 2*num_nodes) over a
+ * vocabulary of `vocab` entries.  The workspace holds per-row partial
+ * normalisers, per-request decisions and per-request completion counters.
+ * It must be 256-byte aligned; it needs no initialisation (each call first
+ * clears its counters on `stream`) and its contents are undefined between
+ * calls.  Two calls that may run concurrently need two workspaces.
+ * Returns 0 for invalid arguments.
+ */
+SPECVERIFY_API size_t spec_verify_workspace_size(int batch, int rows_per_req, int vocab);
+
+/* Static text for a return code (never NULL). */
+SPECVERIFY_API const char *spec_verify_strerror(int code);
+
+/*
+ * Linear stochastic verification.
+ *   target_logits [B][k+1][row_stride]: row j is the target distribution for
+ *                 the token after draft j-1 (row 0: after the committed
+ *                 prefix; row k: the bonus row).
+ *   draft_logits  [B][k][row_stride]: row j is the draft distribution that
+ *                 draft token j was drawn from.
+ *   draft_tokens  [B][k] int32.
+ *   1 <= k <= SPEC_MAX_K, V >= 1, row_stride >= V, temperature > 0 finite.
+ * For each request: n = the first j whose test u_j * q_j(x_j) < p_j(x_j)
+ * fails (u_j = U(seed, b, j, 0, offset)), or k.  If n < k the token at n is
+ * drawn from max(0, p_n - q_n) (renormalised; if that mass is exactly zero,
+ * from p_n); if n == k from p_k, both by inverse CDF with
+ * u = U(seed, b, n, 1, offset): the smallest v whose running sum of weights
+ * exceeds u times the total.
+ * Outputs: out_tokens [B][k+1] = x_0..x_{n-1}, the sampled token, then -1;
+ *          accepted_len [B] = n;
+ *          dbg_logp, dbg_logq [B][k] (nullable, fp32): log p_j(x_j), log q_j(x_j);
+ *          status (nullable, one int32): error bits, OR-ed in.
+ * workspace: at least spec_verify_workspace_size(B, 2k+1, V) bytes.
+ */
+SPECVERIFY_API int spec_verify_linear(const void *target_logits, const void *draft_logits, spec_dtype_t dtype,
+                       int64_t row_stride, const int32_t *draft_tokens, int batch, int k,
+                       int vocab, float temperature, uint64_t seed, uint32_t offset,
+                       int32_t *out_tokens, int32_t *accepted_len, float *dbg_logp,
+                       float *dbg_logq, int32_t *status, void *workspace,
+                       size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Greedy (argmax-match) verification ("Accelerating Sonar through
+ * speculation", section "Target-Draft": the draft emits its top token at
+ * each step).  g_j = argmax_v target_logits[b][j][v] over [0, V), ties to the
+ * lowest index; n = first j < k with draft_tokens[b][j] != g_j, else k.
+ * Outputs: out_tokens [B][k+1] = x_0..x_{n-1}, g_n, then -1; accepted_len [B] = n.
+ * Draft logits are not read and the temperature does not apply.
+ * Needs no workspace: the argmax of a request is merged across a thread-block
+ * cluster in distributed shared memory.
+ */
+SPECVERIFY_API int spec_verify_greedy(const void *target_logits, spec_dtype_t dtype, int64_t row_stride,
+                       const int32_t *draft_tokens, int batch, int k, int vocab,
+                       int32_t *out_tokens, int32_t *accepted_len, int32_t *status,
+                       cudaStream_t stream);
+
+/*
+ * Tree verification ("Accelerating Sonar through speculation", section
+ * "EAGLE": drafts form a tree of top-K candidates; the longest acceptable
+ * sequence is kept and one target token is appended).
+ *   target_logits [B][N][row_stride]: row i = target distribution of the
+ *                 token after node i.
+ *   draft_logits  [B][N][row_stride]: row i = draft distribution node i's
+ *                 children were drawn from; NULL when stochastic == 0; only
+ *                 rows of nodes that have children are read.
+ *   node_tokens   [B][N] int32: token of node i (entry 0, the root, ignored).
+ *   parents       [B][N] int32: parents[0] == -1, 0 <= parents[i] < i.
+ *   1 <= N <= SPEC_MAX_NODES, 1 <= max_depth, every node depth <= max_depth.
+ * Node i >= 1 is accepted when its parent is accepted and its test passes:
+ *   greedy:     node_tokens[i] == argmax(target row parents[i]);
+ *   stochastic: u * q_par(t) < p_par(t) with u = U(seed, b, i-1, 0, offset)
+ *               (position i-1 is the node's draft index, so a chain tree
+ *               draws exactly the numbers of spec_verify_linear).
+ * d = the deepest accepted node, ties to the lowest index (d = 0 when none).
+ * Outputs: out_tokens [B][max_depth+1] = tokens of the nodes on the path
+ *          root->d (root excluded), then a bonus token from target row d
+ *          (greedy: its argmax; stochastic: inverse CDF of p_d with
+ *          u = U(seed, b, d, 1, offset)), then -1;
+ *          accepted_len [B] = depth(d);
+ *          out_path_nodes [B][max_depth+1] (nullable): node at depth 0..depth(d)
+ *          (entry 0 = 0, the root), then -1.
+ * The stochastic tree test has no residual step: it does not keep the
+ * target distribution exactly (a variant that trades the guarantee for
+ * simplicity, as "Speculative decoding explained" allows).
+ * workspace: at least spec_verify_workspace_size(B, 2*N, V) bytes.
+ */
+SPECVERIFY_API int spec_verify_tree(const void *target_logits, const void *draft_logits, spec_dtype_t dtype,
+                     int64_t row_stride, const int32_t *node_tokens, const int32_t *parents,
+                     int batch, int num_nodes, int max_depth, int vocab, int stochastic,
+                     float temperature, uint64_t seed, uint32_t offset, int32_t *out_tokens,
+                     int32_t *accepted_len, int32_t *out_path_nodes, int32_t *status,
+                     void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Diagnostic: the uniforms the kernels draw.  out [batch][count] (device,
+ * double) = U(seed, b, first_position + i, purpose, offset).  Lets a caller
+ * check the device Philox stream against an independent implementation.
+ */
+SPECVERIFY_API int spec_verify_debug_uniforms(uint64_t seed, uint32_t offset, uint32_t purpose, int batch,
+                               int count, int first_position, double *out,
+                               cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPECVERIFY_H */

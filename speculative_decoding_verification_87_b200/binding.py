@@ -1,0 +1,228 @@
+"""ctypes binding of libspecverify.so: argument marshalling only.
+
+Each function takes torch CUDA tensors, checks their shapes and dtypes,
+passes raw device pointers and the current CUDA stream to the C ABI of the
+same name (declared in include/specverify.h) and returns the output
+tensors.  Every step of the computation runs in the library's kernels; there
+is no fallback.  If the library has not been built, the first call raises.
+
+Build it with ``python -m speculative_decoding_verification_87_b200.build``.
+"""
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libspecverify.so")
+
+SPEC_F32, SPEC_BF16 = 0, 1
+SPEC_OK = 0
+STATUS_TOKEN, STATUS_TREE, STATUS_LOGIT = 1, 2, 4
+MAX_K, MAX_NODES = 32, 1024
+SYMBOLS = ("spec_verify_workspace_size", "spec_verify_strerror", "spec_verify_linear",
+           "spec_verify_greedy", "spec_verify_tree", "spec_verify_debug_uniforms")
+
+_lib = None
+_lock = threading.Lock()
+_ws_cache = {}
+
+_P, _I, _I64, _U32, _U64, _F, _SZ = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
+                                     ctypes.c_uint32, ctypes.c_uint64, ctypes.c_float,
+                                     ctypes.c_size_t)
+
+
+class SpecVerifyError(RuntimeError):
+    pass
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libspecverify.so and declare its C signatures."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise SpecVerifyError(
+                f"{path} is missing: build it with "
+                "`python -m speculative_decoding_verification_87_b200.build`")
+        L = ctypes.CDLL(path)
+        L.spec_verify_workspace_size.argtypes = [_I, _I, _I]
+        L.spec_verify_workspace_size.restype = _SZ
+        L.spec_verify_strerror.argtypes = [_I]
+        L.spec_verify_strerror.restype = ctypes.c_char_p
+        L.spec_verify_linear.argtypes = [_P, _P, _I, _I64, _P, _I, _I, _I, _F, _U64, _U32, _P, _P,
+                                         _P, _P, _P, _P, _SZ, _P]
+        L.spec_verify_linear.restype = _I
+        L.spec_verify_greedy.argtypes = [_P, _I, _I64, _P, _I, _I, _I, _P, _P, _P, _P]
+        L.spec_verify_greedy.restype = _I
+        L.spec_verify_tree.argtypes = [_P, _P, _I, _I64, _P, _P, _I, _I, _I, _I, _I, _F, _U64,
+                                       _U32, _P, _P, _P, _P, _P, _SZ, _P]
+        L.spec_verify_tree.restype = _I
+        L.spec_verify_debug_uniforms.argtypes = [_U64, _U32, _U32, _I, _I, _I, _P, _P]
+        L.spec_verify_debug_uniforms.restype = _I
+        _lib = L
+        return L
+
+
+def _check(rc: int, what: str):
+    if rc != SPEC_OK:
+        msg = load_library().spec_verify_strerror(rc).decode()
+        raise SpecVerifyError(f"{what} failed ({rc}): {msg}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SPEC_BF16
+    if t.dtype == torch.float32:
+        return SPEC_F32
+    raise TypeError(f"logits must be bfloat16 or float32, got {t.dtype}")
+
+
+def _need_cuda(name, t, dtype=None, shape=None):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def workspace_size(batch: int, rows_per_req: int, vocab: int) -> int:
+    return int(load_library().spec_verify_workspace_size(batch, rows_per_req, vocab))
+
+
+def workspace(batch: int, rows_per_req: int, vocab: int, device=None) -> torch.Tensor:
+    """A cached uint8 device buffer large enough for the call (256-byte aligned)."""
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    need = workspace_size(batch, rows_per_req, vocab)
+    if need == 0:
+        raise ValueError("invalid workspace request")
+    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    buf = _ws_cache.get(key)
+    if buf is None or buf.numel() < need:
+        buf = torch.empty(need + 256, dtype=torch.uint8, device=device)
+        _ws_cache[key] = buf
+    off = (-buf.data_ptr()) % 256
+    return buf[off:off + need]
+
+
+def spec_verify_linear(target_logits, draft_logits, draft_tokens, vocab, temperature, seed=0,
+                       offset=0, out_tokens=None, accepted_len=None, dbg_logp=None,
+                       dbg_logq=None, status=None, workspace_buf=None, stream=None):
+    """target_logits [B][k+1][stride], draft_logits [B][k][stride] (bf16/fp32),
+    draft_tokens [B][k] int32.  Returns (out_tokens [B][k+1], accepted_len [B])."""
+    _need_cuda("target_logits", target_logits)
+    B, R, stride = target_logits.shape
+    k = R - 1
+    _need_cuda("draft_logits", draft_logits, target_logits.dtype, (B, k, stride))
+    _need_cuda("draft_tokens", draft_tokens, torch.int32, (B, k))
+    dev = target_logits.device
+    if out_tokens is None:
+        out_tokens = torch.empty((B, k + 1), dtype=torch.int32, device=dev)
+    if accepted_len is None:
+        accepted_len = torch.empty((B,), dtype=torch.int32, device=dev)
+    _need_cuda("out_tokens", out_tokens, torch.int32, (B, k + 1))
+    _need_cuda("accepted_len", accepted_len, torch.int32, (B,))
+    for name, t in (("dbg_logp", dbg_logp), ("dbg_logq", dbg_logq)):
+        if t is not None:
+            _need_cuda(name, t, torch.float32, (B, k))
+    if status is not None:
+        _need_cuda("status", status, torch.int32)
+    if workspace_buf is None:
+        workspace_buf = workspace(B, 2 * k + 1, vocab, dev) if B > 0 else None
+    ws_bytes = 0 if workspace_buf is None else workspace_buf.numel()
+    rc = load_library().spec_verify_linear(
+        _ptr(target_logits), _ptr(draft_logits), _dtype_code(target_logits), stride,
+        _ptr(draft_tokens), B, k, vocab, float(temperature), int(seed), int(offset),
+        _ptr(out_tokens), _ptr(accepted_len), _ptr(dbg_logp), _ptr(dbg_logq), _ptr(status),
+        _ptr(workspace_buf), ws_bytes, _stream(stream))
+    _check(rc, "spec_verify_linear")
+    return out_tokens, accepted_len
+
+
+def spec_verify_greedy(target_logits, draft_tokens, vocab, out_tokens=None, accepted_len=None,
+                       status=None, stream=None):
+    """target_logits [B][k+1][stride], draft_tokens [B][k] int32."""
+    _need_cuda("target_logits", target_logits)
+    B, R, stride = target_logits.shape
+    k = R - 1
+    _need_cuda("draft_tokens", draft_tokens, torch.int32, (B, k))
+    dev = target_logits.device
+    if out_tokens is None:
+        out_tokens = torch.empty((B, k + 1), dtype=torch.int32, device=dev)
+    if accepted_len is None:
+        accepted_len = torch.empty((B,), dtype=torch.int32, device=dev)
+    _need_cuda("out_tokens", out_tokens, torch.int32, (B, k + 1))
+    _need_cuda("accepted_len", accepted_len, torch.int32, (B,))
+    if status is not None:
+        _need_cuda("status", status, torch.int32)
+    rc = load_library().spec_verify_greedy(
+        _ptr(target_logits), _dtype_code(target_logits), stride, _ptr(draft_tokens), B, k, vocab,
+        _ptr(out_tokens), _ptr(accepted_len), _ptr(status), _stream(stream))
+    _check(rc, "spec_verify_greedy")
+    return out_tokens, accepted_len
+
+
+def spec_verify_tree(target_logits, draft_logits, node_tokens, parents, max_depth, vocab,
+                     stochastic, temperature=1.0, seed=0, offset=0, out_tokens=None,
+                     accepted_len=None, out_path_nodes=None, status=None, workspace_buf=None,
+                     stream=None):
+    """target_logits [B][N][stride]; draft_logits [B][N][stride] or None (greedy);
+    node_tokens, parents [B][N] int32.  Returns (out_tokens [B][D+1],
+    accepted_len [B], out_path_nodes [B][D+1] or None)."""
+    _need_cuda("target_logits", target_logits)
+    B, N, stride = target_logits.shape
+    if stochastic:
+        _need_cuda("draft_logits", draft_logits, target_logits.dtype, (B, N, stride))
+    _need_cuda("node_tokens", node_tokens, torch.int32, (B, N))
+    _need_cuda("parents", parents, torch.int32, (B, N))
+    dev = target_logits.device
+    W = max_depth + 1
+    if out_tokens is None:
+        out_tokens = torch.empty((B, W), dtype=torch.int32, device=dev)
+    if accepted_len is None:
+        accepted_len = torch.empty((B,), dtype=torch.int32, device=dev)
+    _need_cuda("out_tokens", out_tokens, torch.int32, (B, W))
+    _need_cuda("accepted_len", accepted_len, torch.int32, (B,))
+    if out_path_nodes is not None:
+        _need_cuda("out_path_nodes", out_path_nodes, torch.int32, (B, W))
+    if status is not None:
+        _need_cuda("status", status, torch.int32)
+    if workspace_buf is None:
+        workspace_buf = workspace(B, 2 * N, vocab, dev) if B > 0 else None
+    ws_bytes = 0 if workspace_buf is None else workspace_buf.numel()
+    rc = load_library().spec_verify_tree(
+        _ptr(target_logits), _ptr(draft_logits if stochastic else None),
+        _dtype_code(target_logits), stride, _ptr(node_tokens), _ptr(parents), B, N, max_depth,
+        vocab, int(bool(stochastic)), float(temperature), int(seed), int(offset), _ptr(out_tokens),
+        _ptr(accepted_len), _ptr(out_path_nodes), _ptr(status), _ptr(workspace_buf), ws_bytes,
+        _stream(stream))
+    _check(rc, "spec_verify_tree")
+    return out_tokens, accepted_len, out_path_nodes
+
+
+def spec_verify_debug_uniforms(seed, offset, purpose, batch, count, first_position=0,
+                               device=None, stream=None):
+    """[batch][count] float64 device tensor of the kernels' uniforms."""
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    out = torch.empty((batch, count), dtype=torch.float64, device=device)
+    rc = load_library().spec_verify_debug_uniforms(int(seed), int(offset), int(purpose), batch,
+                                                   count, first_position, _ptr(out),
+                                                   _stream(stream))
+    _check(rc, "spec_verify_debug_uniforms")
+    return out

@@ -1,0 +1,110 @@
+"""The C-ABI library builds for sm_100a, loads without a GPU, exports every
+symbol include/specverify.h declares, and rejects bad arguments on the host
+before touching the device (these calls return before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "specverify.h")
+
+SPEC_OK, SPEC_EINVAL, SPEC_EALIGN, SPEC_EUNSUPPORTED, SPEC_ECUDA, SPEC_EWORKSPACE = 0, -1, -2, -3, -4, -5
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from speculative_decoding_verification_87_b200 import binding, build
+    build.build()
+    return binding.load_library()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return re.findall(r"SPECVERIFY_API\s+[\w\s\*]+?\b(spec_\w+)\s*\(", text)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_symbols())
+    assert {"spec_verify_linear", "spec_verify_greedy", "spec_verify_tree",
+            "spec_verify_workspace_size", "spec_verify_strerror"} <= names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    from speculative_decoding_verification_87_b200 import binding
+    assert set(declared_symbols()) == set(binding.SYMBOLS)
+
+
+def test_workspace_size(lib):
+    a = lib.spec_verify_workspace_size(64, 17, 128256)
+    b = lib.spec_verify_workspace_size(128, 17, 128256)
+    assert a > 0 and b > a and a % 256 == 0
+    assert lib.spec_verify_workspace_size(0, 17, 100) > 0
+    assert lib.spec_verify_workspace_size(4, 0, 100) == 0
+    assert lib.spec_verify_workspace_size(4, 9, 0) == 0
+    assert lib.spec_verify_workspace_size(-1, 9, 10) == 0
+
+
+def test_strerror(lib):
+    for code in (SPEC_OK, SPEC_EINVAL, SPEC_EALIGN, SPEC_EUNSUPPORTED, SPEC_ECUDA,
+                 SPEC_EWORKSPACE, 12345):
+        assert isinstance(lib.spec_verify_strerror(code), bytes)
+    assert lib.spec_verify_strerror(SPEC_OK) == b"ok"
+
+
+def _linear(lib, tl=0x1000, dl=0x2000, dtype=1, stride=128, tokens=0x3000, batch=2, k=3,
+            vocab=100, temperature=1.0, ws=0x10000, ws_bytes=1 << 30):
+    P = ctypes.c_void_p
+    return lib.spec_verify_linear(P(tl), P(dl), dtype, stride, P(tokens), batch, k, vocab,
+                                  temperature, 0, 0, P(0x4000), P(0x5000), None, None, None,
+                                  P(ws), ws_bytes, None)
+
+
+def test_linear_host_validation(lib):
+    assert _linear(lib, k=0) == SPEC_EINVAL
+    assert _linear(lib, k=33) == SPEC_EUNSUPPORTED
+    assert _linear(lib, batch=-1) == SPEC_EINVAL
+    assert _linear(lib, temperature=0.0) == SPEC_EINVAL
+    assert _linear(lib, temperature=float("nan")) == SPEC_EINVAL
+    assert _linear(lib, temperature=float("inf")) == SPEC_EINVAL
+    assert _linear(lib, vocab=0) == SPEC_EINVAL
+    assert _linear(lib, vocab=129) == SPEC_EINVAL            # stride < vocab
+    assert _linear(lib, dtype=7) == SPEC_EINVAL
+    assert _linear(lib, tl=0) == SPEC_EINVAL
+    assert _linear(lib, dl=0) == SPEC_EINVAL
+    assert _linear(lib, tokens=0) == SPEC_EINVAL
+    assert _linear(lib, stride=100) == SPEC_EALIGN           # 200-byte bf16 rows
+    assert _linear(lib, tl=0x1008) == SPEC_EALIGN
+    assert _linear(lib, ws=0) == SPEC_EWORKSPACE
+    assert _linear(lib, ws=0x10010) == SPEC_EWORKSPACE
+    assert _linear(lib, ws_bytes=16) == SPEC_EWORKSPACE
+    assert _linear(lib, batch=0) == SPEC_OK                  # nothing to enqueue
+    assert _linear(lib, batch=0, tl=0, dl=0, tokens=0) == SPEC_OK
+
+
+def test_greedy_and_tree_host_validation(lib):
+    P = ctypes.c_void_p
+    g = lambda **kw: lib.spec_verify_greedy(P(kw.get("tl", 0x1000)), kw.get("dtype", 0),
+                                            kw.get("stride", 64), P(0x2000), kw.get("batch", 3),
+                                            kw.get("k", 2), kw.get("vocab", 50), P(0x3000),
+                                            P(0x4000), None, None)
+    assert g(k=0) == SPEC_EINVAL and g(k=40) == SPEC_EUNSUPPORTED
+    assert g(stride=63) == SPEC_EALIGN and g(vocab=65) == SPEC_EINVAL
+    assert g(batch=0) == SPEC_OK
+
+    def t(**kw):
+        return lib.spec_verify_tree(P(0x1000), P(kw.get("dl", 0x2000)), 1, 64, P(0x3000),
+                                    P(0x3800), kw.get("batch", 2), kw.get("nodes", 60),
+                                    kw.get("depth", 6), 60, kw.get("stoch", 1),
+                                    kw.get("temp", 1.0), 0, 0, P(0x4000), P(0x5000), None, None,
+                                    P(0x10000), kw.get("ws_bytes", 1 << 30), None)
+    assert t(nodes=0) == SPEC_EINVAL and t(nodes=1025) == SPEC_EUNSUPPORTED
+    assert t(depth=0) == SPEC_EINVAL
+    assert t(dl=0) == SPEC_EINVAL                 # stochastic trees read draft rows
+    assert t(dl=0, batch=0) == SPEC_OK            # an empty batch reads nothing
+    assert t(temp=-1.0) == SPEC_EINVAL
+    assert t(ws_bytes=8) == SPEC_EWORKSPACE
+    assert t(batch=0) == SPEC_OK
