@@ -133,6 +133,33 @@ SPECVERIFY_API int spec_verify_linear(const void *target_logits, const void *dra
                        size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * spec_verify_linear without a workspace argument, for callers that cannot
+ * allocate device memory: a plugin whose host framework owns the device
+ * pool and hands out no workspace, or a serving loop that forbids
+ * cudaMalloc once running.  The pages have no counterpart of this call; it
+ * is a packaging convenience.  Inputs, outputs, results and error codes are
+ * those of spec_verify_linear.  Its scratch is one static device array of
+ * SPEC_NOALLOC_SCRATCH_BYTES compiled into the library, which every GPU that
+ * loads the library holds until the process exits; the call itself
+ * allocates nothing.  A request that needs more scratch than that
+ * (spec_verify_workspace_size(B, 2k+1, V) > SPEC_NOALLOC_SCRATCH_BYTES)
+ * returns SPEC_EUNSUPPORTED before anything is enqueued.  The first call on
+ * a device, made with that device current, looks up the array's device
+ * address; make it before any stream capture starts.  All calls on a
+ * device share the array: each clears what must start at zero, but calls
+ * that overlap on the GPU race and must be serialised by the caller.
+ */
+#define SPEC_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+SPECVERIFY_API int spec_verify_linear_noalloc(const void *target_logits, const void *draft_logits,
+                                              spec_dtype_t dtype, int64_t row_stride,
+                                              const int32_t *draft_tokens, int batch, int k,
+                                              int vocab, float temperature, uint64_t seed,
+                                              uint32_t offset, int32_t *out_tokens,
+                                              int32_t *accepted_len, float *dbg_logp,
+                                              float *dbg_logq, int32_t *status,
+                                              cudaStream_t stream);
+
+/*
  * Greedy (argmax-match) verification ("Accelerating Sonar through
  * speculation", section "Target-Draft": the draft emits its top token at
  * each step).  g_j = argmax_v target_logits[b][j][v] over [0, V), ties to the

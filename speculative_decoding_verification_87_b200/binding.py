@@ -22,7 +22,9 @@ SPEC_OK = 0
 STATUS_TOKEN, STATUS_TREE, STATUS_LOGIT = 1, 2, 4
 MAX_K, MAX_NODES = 32, 1024
 SYMBOLS = ("spec_verify_workspace_size", "spec_verify_strerror", "spec_verify_linear",
-           "spec_verify_greedy", "spec_verify_tree", "spec_verify_debug_uniforms")
+           "spec_verify_greedy", "spec_verify_tree", "spec_verify_debug_uniforms",
+           "spec_verify_linear_noalloc")
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 _lib = None
 _lock = threading.Lock()
@@ -62,6 +64,9 @@ def load_library(path: str = LIB_PATH):
         L.spec_verify_tree.restype = _I
         L.spec_verify_debug_uniforms.argtypes = [_U64, _U32, _U32, _I, _I, _I, _P, _P]
         L.spec_verify_debug_uniforms.restype = _I
+        L.spec_verify_linear_noalloc.argtypes = [_P, _P, _I, _I64, _P, _I, _I, _I, _F, _U64, _U32,
+                                                 _P, _P, _P, _P, _P, _P]
+        L.spec_verify_linear_noalloc.restype = _I
         _lib = L
         return L
 
@@ -226,3 +231,35 @@ def spec_verify_debug_uniforms(seed, offset, purpose, batch, count, first_positi
                                                    _stream(stream))
     _check(rc, "spec_verify_debug_uniforms")
     return out
+
+
+def spec_verify_linear_noalloc(target_logits, draft_logits, draft_tokens, vocab, temperature,
+                               seed, offset, out_tokens, accepted_len, dbg_logp=None,
+                               dbg_logq=None, status=None, stream=None):
+    """Linear verification through the entry point that allocates nothing.
+
+    For callers that cannot allocate device memory (a plugin whose host
+    framework owns the device pool, a serving loop that forbids cudaMalloc
+    while running): the outputs must be passed in, no workspace is taken,
+    and the library uses its own static 8 MiB device scratch.  Calls that
+    overlap on the GPU share that scratch and must not be issued
+    concurrently."""
+    _need_cuda("target_logits", target_logits)
+    B, R, stride = target_logits.shape
+    k = R - 1
+    _need_cuda("draft_logits", draft_logits, target_logits.dtype, (B, k, stride))
+    _need_cuda("draft_tokens", draft_tokens, torch.int32, (B, k))
+    _need_cuda("out_tokens", out_tokens, torch.int32, (B, k + 1))
+    _need_cuda("accepted_len", accepted_len, torch.int32, (B,))
+    for name, t in (("dbg_logp", dbg_logp), ("dbg_logq", dbg_logq)):
+        if t is not None:
+            _need_cuda(name, t, torch.float32, (B, k))
+    if status is not None:
+        _need_cuda("status", status, torch.int32)
+    rc = load_library().spec_verify_linear_noalloc(
+        _ptr(target_logits), _ptr(draft_logits), _dtype_code(target_logits), stride,
+        _ptr(draft_tokens), B, k, vocab, float(temperature), int(seed), int(offset),
+        _ptr(out_tokens), _ptr(accepted_len), _ptr(dbg_logp), _ptr(dbg_logq), _ptr(status),
+        _stream(stream))
+    _check(rc, "spec_verify_linear_noalloc")
+    return out_tokens, accepted_len

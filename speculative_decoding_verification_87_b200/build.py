@@ -2,8 +2,8 @@
 
     python -m speculative_decoding_verification_87_b200.build [--force]
 
-The library is one translation unit (csrc/specverify.cu plus its headers),
-compiled for sm_100a only, with static cudart and -lineinfo.
+The library is built from csrc/*.cu (specverify.cu with its headers, and
+noalloc.cu), compiled for sm_100a only, with static cudart and -lineinfo.
 """
 import glob
 import os
@@ -35,7 +35,8 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if (not force and os.path.exists(LIB)
             and os.path.getmtime(LIB) >= max(os.path.getmtime(s) for s in srcs)):
         return LIB
-    cmd = [NVCC, *NVCC_FLAGS, *extra, "-o", LIB + ".tmp", os.path.join(CSRC, "specverify.cu")]
+    cmd = [NVCC, *NVCC_FLAGS, *extra, "-o", LIB + ".tmp",
+           *sorted(glob.glob(os.path.join(CSRC, "*.cu")))]
     if verbose:
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)
