@@ -217,11 +217,11 @@ class Runner:
             self.parents = dev(w.parents)
             W = w.max_depth + 1
             self.out = torch.empty((w.batch, W), dtype=torch.int32, device=device)
-            self.kernels_per_call = 1 if name == "tree" else 2
+            self.kernels_per_call = 1
         else:
             self.tokens = dev(w.tokens.astype(np.int32))
             self.out = torch.empty((w.batch, w.k + 1), dtype=torch.int32, device=device)
-            self.kernels_per_call = {"greedy": 1}.get(name, 3)
+            self.kernels_per_call = 1
         self.acc = torch.empty((w.batch,), dtype=torch.int32, device=device)
 
     def call(self, offset, target=None, draft=None, tokens=None):

@@ -81,8 +81,11 @@ enum {
     SPEC_STATUS_TOKEN = 1,   /* a draft or node token outside [0, V)                     */
     SPEC_STATUS_TREE = 2,    /* parents[0] != -1, parents[i] not in [0, i), or a node
                                 deeper than max_depth                                    */
-    SPEC_STATUS_LOGIT = 4    /* a NaN logit, or a row with no finite normaliser
+    SPEC_STATUS_LOGIT = 4,   /* a NaN logit, or a row with no finite normaliser
                                 (+inf present, or every entry -inf)                      */
+    SPEC_STATUS_TIMEOUT = 8  /* an idle worker stopped polling for work after its bound
+                                (about a second): requests not yet complete have
+                                undefined outputs.  Not expected in normal operation.   */
 };
 
 /* Limits checked on the host. */
@@ -219,6 +222,17 @@ SPECVERIFY_API int spec_verify_tree(const void *target_logits, const void *draft
 SPECVERIFY_API int spec_verify_debug_uniforms(uint64_t seed, uint32_t offset, uint32_t purpose, int batch,
                                int count, int first_position, double *out,
                                cudaStream_t stream);
+
+/*
+ * Diagnostic: the kernels' base-2 exponentials, out[i] = 2^z[i] for
+ * z[i] <= 0 (device arrays of n doubles).  kind 0: fp64, table driven
+ * (Tang's method; results below 2^-1020 are 0); kind 1: fp32 polynomial on
+ * the FMA pipe (input rounded to fp32; results below 2^-125 are 0);
+ * kind 2: fp32 special-function unit (ex2.approx).  Lets a caller check
+ * their accuracy.
+ */
+SPECVERIFY_API int spec_verify_debug_exp2(const double *z, double *out, int n, int kind,
+                                          cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -19,11 +19,11 @@ LIB_PATH = os.path.join(_HERE, "libspecverify.so")
 
 SPEC_F32, SPEC_BF16 = 0, 1
 SPEC_OK = 0
-STATUS_TOKEN, STATUS_TREE, STATUS_LOGIT = 1, 2, 4
+STATUS_TOKEN, STATUS_TREE, STATUS_LOGIT, STATUS_TIMEOUT = 1, 2, 4, 8
 MAX_K, MAX_NODES = 32, 1024
 SYMBOLS = ("spec_verify_workspace_size", "spec_verify_strerror", "spec_verify_linear",
            "spec_verify_greedy", "spec_verify_tree", "spec_verify_debug_uniforms",
-           "spec_verify_linear_noalloc")
+           "spec_verify_linear_noalloc", "spec_verify_debug_exp2")
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 _lib = None
@@ -67,6 +67,8 @@ def load_library(path: str = LIB_PATH):
         L.spec_verify_linear_noalloc.argtypes = [_P, _P, _I, _I64, _P, _I, _I, _I, _F, _U64, _U32,
                                                  _P, _P, _P, _P, _P, _P]
         L.spec_verify_linear_noalloc.restype = _I
+        L.spec_verify_debug_exp2.argtypes = [_P, _P, _I, _I, _P]
+        L.spec_verify_debug_exp2.restype = _I
         _lib = L
         return L
 
@@ -230,6 +232,18 @@ def spec_verify_debug_uniforms(seed, offset, purpose, batch, count, first_positi
                                                    count, first_position, _ptr(out),
                                                    _stream(stream))
     _check(rc, "spec_verify_debug_uniforms")
+    return out
+
+
+def spec_verify_debug_exp2(z, kind=0, stream=None):
+    """2^z (z <= 0) from one of the kernels' exponentials (kind 0: fp64
+    table driven; 1: fp32 FMA-pipe polynomial; 2: fp32 special-function
+    unit); z a float64 CUDA tensor."""
+    _need_cuda("z", z, torch.float64)
+    out = torch.empty_like(z)
+    rc = load_library().spec_verify_debug_exp2(_ptr(z), _ptr(out), z.numel(), int(kind),
+                                               _stream(stream))
+    _check(rc, "spec_verify_debug_exp2")
     return out
 
 

@@ -1,13 +1,13 @@
-// specverify.cu -- kernels and C ABI of libspecverify.so (sm_100a).
+// specverify.cu -- C ABI of libspecverify.so (sm_100a) and its launches.
 //
-// Call flow of spec_verify_linear (all on the caller's stream, no host sync):
-//   memset(counters) -> k_pass1 (one streaming read of the 2k+1 rows of every
-//   request; the last block of each request decides n) -> k_pass2a (fp64
-//   normalisers of the residual row pair) -> k_pass2b (fp64 segment weights;
-//   the last block of each request draws the token).
-// spec_verify_tree: memset -> k_pass1 (tree decide) [-> k_pass2b if stochastic].
-// spec_verify_greedy: k_greedy_cluster alone (no workspace).
+// spec_verify_linear / spec_verify_tree: one memset of the work counters and
+// one launch of the persistent engine (sv_engine.cuh) on the caller's
+// stream; no host synchronisation.
+// spec_verify_greedy: one launch of the cluster kernel (sv_greedy.cuh); no
+// workspace.
+#include <algorithm>
 #include <climits>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -16,61 +16,12 @@
 
 #include "../../include/specverify.h"
 #include "sv_common.cuh"
-#include "sv_decide.cuh"
+#include "sv_engine.cuh"
+#include "sv_exp64.cuh"
 #include "sv_greedy.cuh"
 #include "sv_philox.cuh"
-#include "sv_sample.cuh"
-#include "sv_stats.cuh"
 
 namespace sv {
-
-template <class Tag, int MODE, int U>
-__global__ void __launch_bounds__(kThreads) k_pass1(const Params p)
-{
-    __shared__ float redf[kWarps];
-    __shared__ int redi[kWarps];
-    const int64_t item = blockIdx.x;
-    const int s = static_cast<int>(item % p.S);
-    const int64_t br = item / p.S;
-    const int r = static_cast<int>(br % p.R);
-    const int b = static_cast<int>(br / p.R);
-    constexpr int kEsz = sizeof(typename Tag::elem);
-
-    const void *base;
-    int64_t row_index;
-    bool active = true;
-    if (MODE == kLinear) {
-        if (r <= p.k) {
-            base = p.tl;
-            row_index = static_cast<int64_t>(b) * (p.k + 1) + r;
-        } else {
-            base = p.dl;
-            row_index = static_cast<int64_t>(b) * p.k + (r - p.k - 1);
-        }
-    } else if (r < p.N) {
-        base = p.tl;
-        row_index = static_cast<int64_t>(b) * p.N + r;
-    } else {
-        base = p.dl;
-        row_index = static_cast<int64_t>(b) * p.N + (r - p.N);
-        active = node_has_child(p, b, r - p.N);
-    }
-    if (active) {
-        const char *row = static_cast<const char *>(base) + row_index * p.stride * kEsz;
-        const int seg_begin = s * p.seg;
-        const int seg_end = min(p.V, seg_begin + p.seg);
-        uint4 raw[U];
-        load_segment<Tag, U>(row, seg_begin, seg_end, raw);
-        float2 part;
-        if (MODE == kTreeGreedy) part = segment_argmax_partial<Tag, U>(raw, seg_begin, redf, redi);
-        else part = segment_softmax_partial<Tag, U>(raw, p.c, redf);
-        if (threadIdx.x == 0) p.rowpart[br * p.S + s] = part;
-    }
-    if (arrive_last(&p.cnt1[b], static_cast<unsigned>(p.R * p.S))) {
-        if (MODE == kLinear) decide_linear<Tag>(p, b);
-        else decide_tree<Tag, MODE>(p, b);
-    }
-}
 
 __global__ void k_debug_uniforms(uint64_t seed, uint32_t offset, uint32_t purpose, int batch,
                                  int count, int first, double *out)
@@ -82,19 +33,34 @@ __global__ void k_debug_uniforms(uint64_t seed, uint32_t offset, uint32_t purpos
                             offset);
 }
 
+__global__ void k_debug_exp2(const double *z, double *out, int n, int kind, Params p)
+{
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    Exp2Table tab;
+    tab.lo = p.exp2tab[threadIdx.x & 31];
+    tab.hi = p.exp2tab[(threadIdx.x & 31) + 32];
+    const double zi = i < n ? z[i] : 0.0;
+    const double v = exp2_fp64(zi, tab);  // every lane calls (warp-collective)
+    if (i < n) {
+        if (kind == 1) out[i] = f32_to_f64(ex2_fma(static_cast<float>(zi)));
+        else if (kind == 2) out[i] = f32_to_f64(ex2_approx(static_cast<float>(zi)));
+        else out[i] = v;
+    }
+}
+
 // ------------------------------------------------------------ host helpers
 namespace {
 
 constexpr size_t kAlign = 256;
-constexpr int kMinSeg = kThreads * F32::kVec;  // smallest pass-1 segment (fp32, U = 1)
+constexpr int kBatchF32 = 32 * 4 * F32::kVec;  // smallest pass-1 segment (fp32, one warp batch)
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-// Workspace layout; counters first.  Region sizes use the smallest pass-1
-// segment, so any per-call segment choice fits.
+// Workspace layout; the counters (cleared per call) come first.  Region
+// sizes use the smallest pass-1 segment, so any per-call choice fits.
 struct Layout {
-    size_t cnt, rowpart, rowstat, req, p2a, p2b, total;
+    size_t ctr, rowpart, rowstat, req, p2part, p2amb, ambbits, p2w, p2lane, total, clear_bytes;
     bool ok;
 };
 
@@ -103,21 +69,29 @@ Layout layout(int B, int R, int V)
     Layout L{};
     L.ok = false;
     if (B < 0 || R < 1 || V < 1) return L;
-    const int64_t smax = ceil_div(V, kMinSeg);
+    const int64_t smax = ceil_div(V, kBatchF32);
     const int64_t s2 = ceil_div(V, kSeg2);
+    const int64_t w32 = ceil_div(V, 32);
     size_t off = 0;
-    L.cnt = off;
-    off = align_up(off + sizeof(unsigned) * 3 * static_cast<size_t>(B));
+    L.ctr = off;
+    L.clear_bytes = sizeof(Counters) + sizeof(unsigned) * (3 + static_cast<size_t>(R)) * static_cast<size_t>(B);
+    off = align_up(off + L.clear_bytes);
     L.rowpart = off;
     off = align_up(off + sizeof(float2) * static_cast<size_t>(B) * R * smax);
     L.rowstat = off;
     off = align_up(off + sizeof(RowStat) * static_cast<size_t>(B) * R);
     L.req = off;
     off = align_up(off + sizeof(ReqInfo) * static_cast<size_t>(B));
-    L.p2a = off;
-    off = align_up(off + sizeof(double2) * static_cast<size_t>(B) * s2);
-    L.p2b = off;
+    L.p2part = off;
+    off = align_up(off + sizeof(double4) * static_cast<size_t>(B) * s2);
+    L.p2amb = off;
+    off = align_up(off + sizeof(int) * static_cast<size_t>(B) * s2);
+    L.ambbits = off;
+    off = align_up(off + sizeof(unsigned) * static_cast<size_t>(B) * w32);
+    L.p2w = off;
     off = align_up(off + sizeof(double) * static_cast<size_t>(B) * s2);
+    L.p2lane = off;
+    off = align_up(off + sizeof(double2) * 32 * static_cast<size_t>(B) * s2);
     L.total = off < kAlign ? kAlign : off;
     L.ok = true;
     return L;
@@ -145,58 +119,98 @@ int check_rows(const void *tl, const void *dl, bool need_dl)
     return SPEC_OK;
 }
 
-// Pass-1 vectors per thread: enough blocks to fill the GPU several times.
-int choose_u(int B, int R, int V, int vec)
-{
-    for (int u : {4, 2}) {
-        const int64_t S = ceil_div(V, static_cast<int64_t>(kThreads) * vec * u);
-        if (static_cast<int64_t>(B) * R * S >= 2048) return u;
-    }
-    return 1;
-}
-
 void fill_workspace(Params &p, void *ws, const Layout &L)
 {
     char *w = static_cast<char *>(ws);
-    auto *cnt = reinterpret_cast<unsigned *>(w + L.cnt);
-    p.cnt1 = cnt;
-    p.cnt2a = cnt + p.B;
-    p.cnt2b = cnt + 2 * static_cast<int64_t>(p.B);
+    p.ctr = reinterpret_cast<Counters *>(w + L.ctr);
+    auto *per_req = reinterpret_cast<unsigned *>(w + L.ctr + sizeof(Counters));
+    p.a_done = per_req;
+    p.p2_done = per_req + p.B;
+    p.decided = per_req + 2 * static_cast<int64_t>(p.B);
+    p.row_done = per_req + 3 * static_cast<int64_t>(p.B);
     p.rowpart = reinterpret_cast<float2 *>(w + L.rowpart);
     p.rowstat = reinterpret_cast<RowStat *>(w + L.rowstat);
     p.req = reinterpret_cast<ReqInfo *>(w + L.req);
-    p.p2a = reinterpret_cast<double2 *>(w + L.p2a);
-    p.p2b = reinterpret_cast<double *>(w + L.p2b);
+    p.p2part = reinterpret_cast<double4 *>(w + L.p2part);
+    p.p2amb = reinterpret_cast<int *>(w + L.p2amb);
+    p.ambbits = reinterpret_cast<unsigned *>(w + L.ambbits);
+    p.p2w = reinterpret_cast<double *>(w + L.p2w);
+    p.p2lane = reinterpret_cast<double2 *>(w + L.p2lane);
 }
+
+// 2^(j/64), j = 0..63, from the host math library.
+void fill_exp2_table(Params &p)
+{
+    for (int j = 0; j < 64; ++j) p.exp2tab[j] = std::exp2(static_cast<double>(j) / 64.0);
+}
+
+// Pass-1 segment: the largest of 4, 2, 1 warp batches that still gives
+// every worker several items.
+int choose_seg(int B, int R, int V, spec_dtype_t dtype, int64_t min_items)
+{
+    const int batch = 32 * 4 * vec_of(dtype);
+    for (int nb : {4, 2}) {
+        const int64_t S = ceil_div(V, static_cast<int64_t>(batch) * nb);
+        if (static_cast<int64_t>(B) * R * S >= min_items) return batch * nb;
+    }
+    return batch;
+}
+
+// Engine occupancy per device and instantiation.
+std::mutex g_mu;
+int g_engine_blocks[64][2][3];
+int g_sm_count[64];
 
 template <class Tag, int MODE>
-cudaError_t launch_pass1(const Params &p, int U, cudaStream_t st)
+int engine_blocks_per_sm(int dev, int dtype_index)
 {
-    const unsigned grid = static_cast<unsigned>(static_cast<int64_t>(p.B) * p.R * p.S);
-    switch (U) {
-    case 4: k_pass1<Tag, MODE, 4><<<grid, kThreads, 0, st>>>(p); break;
-    case 2: k_pass1<Tag, MODE, 2><<<grid, kThreads, 0, st>>>(p); break;
-    default: k_pass1<Tag, MODE, 1><<<grid, kThreads, 0, st>>>(p); break;
-    }
-    return cudaGetLastError();
+    int &slot = g_engine_blocks[dev][dtype_index][MODE];
+    if (slot > 0) return slot;
+    if (cudaFuncSetAttribute(k_engine<Tag, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kRingBytes)) != cudaSuccess)
+        return -1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_engine<Tag, MODE>, kThreads, kRingBytes) !=
+            cudaSuccess ||
+        n < 1)
+        return -1;
+    slot = n;
+    return n;
 }
 
-template <class Tag>
-cudaError_t launch_pass2(const Params &p, bool with_2a, cudaStream_t st)
+int sm_count(int dev)
 {
-    const unsigned grid = static_cast<unsigned>(static_cast<int64_t>(p.B) * p.S2);
-    if (with_2a) {
-        k_pass2a<Tag><<<grid, kThreads, 0, st>>>(p);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
+    int &slot = g_sm_count[dev];
+    if (slot > 0) return slot;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+        return -1;
+    slot = n;
+    return n;
+}
+
+// Clear the counters and launch the engine.
+template <class Tag, int MODE>
+int launch_engine(Params &p, const Layout &L, void *ws, int dtype_index, cudaStream_t st)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SPEC_ECUDA;
+    int per_sm, sms;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        per_sm = engine_blocks_per_sm<Tag, MODE>(dev, dtype_index);
+        sms = sm_count(dev);
     }
-    k_pass2b<Tag><<<grid, kThreads, 0, st>>>(p);
-    return cudaGetLastError();
+    if (per_sm < 1 || sms < 1) return SPEC_ECUDA;
+    const int64_t want = ceil_div(static_cast<int64_t>(p.nA) + p.nP, kWarps - kP2Warps);
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(static_cast<int64_t>(per_sm) * sms, want));
+    if (cudaMemsetAsync(ws, 0, L.clear_bytes, st) != cudaSuccess) return SPEC_ECUDA;
+    k_engine<Tag, MODE><<<static_cast<unsigned>(blocks), kThreads, kRingBytes, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ECUDA;
 }
 
 // Largest number of co-resident greedy clusters, per device and dtype.
 constexpr int kGreedyCluster = 8;
-std::mutex g_mu;
 int g_max_clusters[64][2];
 
 template <class Tag>
@@ -262,10 +276,30 @@ void base_params(Params &p, const void *tl, const void *dl, int64_t stride, int 
     p.V = V;
     const double t = static_cast<double>(T);
     p.inv_t = 1.0 / t;
-    p.c = static_cast<float>(1.4426950408889634 / t);  // log2(e) / T
+    p.c64 = 1.4426950408889634074 / t;  // log2(e) / T
+    p.c = static_cast<float>(p.c64);
     p.seed = seed;
     p.offset = offset;
     p.S2 = static_cast<int>(ceil_div(V, kSeg2));
+    p.W32 = static_cast<int>(ceil_div(V, 32));
+    fill_exp2_table(p);
+}
+
+// Items per request and segment choice shared by the linear and tree calls.
+int setup_items(Params &p, int R, spec_dtype_t dtype, bool pass2)
+{
+    p.R = R;
+    p.seg = choose_seg(p.B, R, p.V, dtype, 16384);
+    p.S = static_cast<int>(ceil_div(p.V, p.seg));
+    const int64_t nA = static_cast<int64_t>(p.B) * R * p.S;
+    const int64_t nP = pass2 ? static_cast<int64_t>(p.B) * p.S2 : 0;
+    if (nA >= (int64_t(1) << 31) || nP >= (int64_t(1) << 31)) return SPEC_EUNSUPPORTED;
+    p.nA = static_cast<unsigned>(nA);
+    p.nP = static_cast<unsigned>(nP);
+    p.div_req = make_fastdiv(static_cast<uint32_t>(R) * static_cast<uint32_t>(p.S));
+    p.div_s = make_fastdiv(static_cast<uint32_t>(p.S));
+    p.div_s2 = make_fastdiv(static_cast<uint32_t>(p.S2));
+    return SPEC_OK;
 }
 
 }  // namespace
@@ -315,40 +349,22 @@ extern "C" int spec_verify_linear(const void *target_logits, const void *draft_l
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 ||
         workspace_bytes < L.total)
         return SPEC_EWORKSPACE;
-    const int vec = vec_of(dtype);
-    const int U = choose_u(batch, R, vocab, vec);
-    const int seg = kThreads * vec * U;
-    const int64_t S = ceil_div(vocab, seg);
-    if (static_cast<int64_t>(batch) * R * S > INT_MAX ||
-        static_cast<int64_t>(batch) * ceil_div(vocab, kSeg2) > INT_MAX)
-        return SPEC_EUNSUPPORTED;
+    if (static_cast<int64_t>(batch) * (k + 1) > INT_MAX) return SPEC_EUNSUPPORTED;
 
     Params p;
     base_params(p, target_logits, draft_logits, row_stride, batch, vocab, temperature, seed, offset);
     p.tokens = draft_tokens;
     p.k = k;
-    p.R = R;
-    p.S = static_cast<int>(S);
-    p.seg = seg;
     p.out = out_tokens;
     p.acc = accepted_len;
     p.dbg_lp = dbg_logp;
     p.dbg_lq = dbg_logq;
     p.status = status;
+    rc = setup_items(p, R, dtype, true);
+    if (rc != SPEC_OK) return rc;
     fill_workspace(p, workspace, L);
-
-    if (cudaMemsetAsync(p.cnt1, 0, sizeof(unsigned) * 3 * static_cast<size_t>(batch), stream) !=
-        cudaSuccess)
-        return SPEC_ECUDA;
-    cudaError_t e;
-    if (dtype == SPEC_BF16) {
-        e = launch_pass1<Bf16, kLinear>(p, U, stream);
-        if (e == cudaSuccess) e = launch_pass2<Bf16>(p, true, stream);
-    } else {
-        e = launch_pass1<F32, kLinear>(p, U, stream);
-        if (e == cudaSuccess) e = launch_pass2<F32>(p, true, stream);
-    }
-    return e == cudaSuccess ? SPEC_OK : SPEC_ECUDA;
+    return dtype == SPEC_BF16 ? launch_engine<Bf16, kLinear>(p, L, workspace, 1, stream)
+                              : launch_engine<F32, kLinear>(p, L, workspace, 0, stream);
 }
 
 extern "C" int spec_verify_greedy(const void *target_logits, spec_dtype_t dtype,
@@ -398,14 +414,7 @@ extern "C" int spec_verify_tree(const void *target_logits, const void *draft_log
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 ||
         workspace_bytes < L.total)
         return SPEC_EWORKSPACE;
-    const int vec = vec_of(dtype);
-    const int U = choose_u(batch, R, vocab, vec);
-    const int seg = kThreads * vec * U;
-    const int64_t S = ceil_div(vocab, seg);
-    if (static_cast<int64_t>(batch) * R * S > INT_MAX ||
-        static_cast<int64_t>(batch) * ceil_div(vocab, kSeg2) > INT_MAX ||
-        static_cast<int64_t>(batch) * (max_depth + 1) > INT_MAX)
-        return SPEC_EUNSUPPORTED;
+    if (static_cast<int64_t>(batch) * (max_depth + 1) > INT_MAX) return SPEC_EUNSUPPORTED;
 
     Params p;
     base_params(p, target_logits, draft_logits, row_stride, batch, vocab,
@@ -414,29 +423,18 @@ extern "C" int spec_verify_tree(const void *target_logits, const void *draft_log
     p.parents = parents;
     p.N = num_nodes;
     p.max_depth = max_depth;
-    p.R = R;
-    p.S = static_cast<int>(S);
-    p.seg = seg;
     p.out = out_tokens;
     p.acc = accepted_len;
     p.path = out_path_nodes;
     p.status = status;
+    rc = setup_items(p, R, dtype, stochastic != 0);
+    if (rc != SPEC_OK) return rc;
     fill_workspace(p, workspace, L);
-
-    if (cudaMemsetAsync(p.cnt1, 0, sizeof(unsigned) * 3 * static_cast<size_t>(batch), stream) !=
-        cudaSuccess)
-        return SPEC_ECUDA;
-    cudaError_t e;
-    if (dtype == SPEC_BF16) {
-        e = stochastic ? launch_pass1<Bf16, kTreeStochastic>(p, U, stream)
-                       : launch_pass1<Bf16, kTreeGreedy>(p, U, stream);
-        if (e == cudaSuccess && stochastic) e = launch_pass2<Bf16>(p, false, stream);
-    } else {
-        e = stochastic ? launch_pass1<F32, kTreeStochastic>(p, U, stream)
-                       : launch_pass1<F32, kTreeGreedy>(p, U, stream);
-        if (e == cudaSuccess && stochastic) e = launch_pass2<F32>(p, false, stream);
-    }
-    return e == cudaSuccess ? SPEC_OK : SPEC_ECUDA;
+    if (dtype == SPEC_BF16)
+        return stochastic ? launch_engine<Bf16, kTreeStochastic>(p, L, workspace, 1, stream)
+                          : launch_engine<Bf16, kTreeGreedy>(p, L, workspace, 1, stream);
+    return stochastic ? launch_engine<F32, kTreeStochastic>(p, L, workspace, 0, stream)
+                      : launch_engine<F32, kTreeGreedy>(p, L, workspace, 0, stream);
 }
 
 extern "C" int spec_verify_debug_uniforms(uint64_t seed, uint32_t offset, uint32_t purpose,
@@ -450,5 +448,18 @@ extern "C" int spec_verify_debug_uniforms(uint64_t seed, uint32_t offset, uint32
     if (blocks > INT_MAX) return SPEC_EUNSUPPORTED;
     k_debug_uniforms<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(seed, offset, purpose, batch,
                                                                          count, first_position, out);
+    return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ECUDA;
+}
+
+extern "C" int spec_verify_debug_exp2(const double *z, double *out, int n, int kind,
+                                      cudaStream_t stream)
+{
+    if (n < 0 || (n > 0 && (!z || !out)) || kind < 0 || kind > 2) return SPEC_EINVAL;
+    if (n == 0) return SPEC_OK;
+    Params p;
+    std::memset(&p, 0, sizeof p);
+    fill_exp2_table(p);
+    const int blocks = static_cast<int>(ceil_div(n, 256));
+    k_debug_exp2<<<blocks, 256, 0, stream>>>(z, out, n, kind, p);
     return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ECUDA;
 }

@@ -15,14 +15,14 @@ constexpr int kWarps = kThreads / 32;
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
 // Per-request status bits (mirror SPEC_STATUS_* in the public header).
-enum : int { kStToken = 1, kStTree = 2, kStLogit = 4 };
+enum : int { kStToken = 1, kStTree = 2, kStLogit = 4, kStTimeout = 8 };
 
 // Philox counter purposes.
 enum : uint32_t { kPurposeAccept = 0, kPurposeSample = 1 };
 
-// Pass-2 segment: 4096 vocabulary entries, 16 contiguous entries per thread.
-constexpr int kSeg2 = 4096;
-constexpr int kPerThread2 = kSeg2 / kThreads;
+// Pass-2 segment: 2048 vocabulary entries, 64 contiguous entries per lane.
+constexpr int kSeg2 = 2048;
+constexpr int kLane2 = kSeg2 / 32;
 
 // Storage tags: element type and entries per 16-byte vector.
 struct Bf16 {
@@ -45,6 +45,81 @@ __device__ __forceinline__ float ex2_approx(float x)
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x for x <= 0 on the FMA pipe: round x to the nearest integer n with the
+// 1.5 * 2^23 shift, evaluate 2^f (f = x - n in [-1/2, 1/2]) by its Taylor
+// polynomial of degree 6 (sum (f ln 2)^k / k!, truncation below 1.2e-7
+// relative) and add n to the exponent field.  Results below 2^-125 are 0.
+// Used for part of the pass-1 exponentials so that the special-function
+// unit, which the rest can saturate, is not the limit.
+constexpr float kF1 = 0.693147180559945309f;
+constexpr float kF2 = 0.240226506959100712f;
+constexpr float kF3 = 0.0555041086648215800f;
+constexpr float kF4 = 0.00961812910762847716f;
+constexpr float kF5 = 0.00133335581464284434f;
+constexpr float kF6 = 0.000154035303933816099f;
+__device__ __forceinline__ float ex2_fma(float x)
+{
+    const float xc = fmaxf(x, -125.0f);
+    const float t = __fadd_rn(xc, 12582912.0f);  // 1.5 * 2^23
+    const float f = xc - __fadd_rn(t, -12582912.0f);
+    float q = fmaf(kF6, f, kF5);
+    q = fmaf(q, f, kF4);
+    q = fmaf(q, f, kF3);
+    q = fmaf(q, f, kF2);
+    q = fmaf(q, f, kF1);
+    q = fmaf(q, f, 1.0f);
+    const int n = __float_as_int(t) - 0x4B400000;
+    const float r = __int_as_float(__float_as_int(q) + (n << 23));
+    return x < -125.0f ? 0.0f : r;
+}
+
+// Exact float -> double widening with integer operations only (no
+// conversion instruction); subnormal floats become signed zero, which no
+// fp64 quantity here can tell apart from them.
+__device__ __forceinline__ double f32_to_f64(float v)
+{
+    const uint32_t u = __float_as_uint(v);
+    const uint32_t sign = u & 0x80000000u;
+    const uint32_t e = (u >> 23) & 0xFFu;
+    const uint32_t m = u & 0x7FFFFFu;
+    uint32_t hi, lo;
+    if (e == 0xFFu) {
+        hi = sign | 0x7FF00000u | (m >> 3);
+        lo = m << 29;
+    } else if (e == 0u) {
+        hi = sign;
+        lo = 0u;
+    } else {
+        hi = sign | ((e + 896u) << 20) | (m >> 3);
+        lo = m << 29;
+    }
+    return __hiloint2double(static_cast<int>(hi), static_cast<int>(lo));
+}
+
+// n / d and n % d for a divisor fixed per launch, by multiply-high and
+// shift (no division instruction): with l = ceil(log2 d) and
+// m = floor(2^(32+l) / d) + 1, q = (n * m) >> (32 + l) is exact for
+// n, d < 2^31.
+struct FastDiv {
+    uint32_t d;
+    uint32_t shift;
+    uint64_t m;
+};
+__host__ __device__ inline FastDiv make_fastdiv(uint32_t d)
+{
+    FastDiv f;
+    f.d = d;
+    uint32_t l = 0;
+    while ((1ull << l) < d) ++l;
+    f.shift = 32 + l;
+    f.m = ((1ull << (32 + l)) / d) + 1;
+    return f;
+}
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv &f)
+{
+    return static_cast<uint32_t>((static_cast<uint64_t>(n) * f.m) >> f.shift);
 }
 
 // max that returns NaN when either input is NaN (a NaN logit must poison
@@ -136,6 +211,20 @@ __device__ __forceinline__ float vec_max<F32>(uint4 v)
 {
     return max_nan(max_nan(__uint_as_float(v.x), __uint_as_float(v.y)),
                    max_nan(__uint_as_float(v.z), __uint_as_float(v.w)));
+}
+
+// Argmax combine: larger value wins, ties go to the lower index.
+__device__ __forceinline__ void argmax_take(float &bv, int &bi, float ov, int oi)
+{
+    if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+    }
+}
+
+__device__ __forceinline__ unsigned ld_volatile(const unsigned *p)
+{
+    return *reinterpret_cast<const volatile unsigned *>(p);
 }
 
 // ---------------------------------------------------------------- reductions
@@ -241,20 +330,28 @@ struct RowStat {
     double s;  // stochastic: sum_v exp((l_v - m) / T)
 };
 
-// What pass 2 must do for one request.
+// What the final draw of one request needs.
 enum : int { kModeNone = 0, kModeTargetRow = 1, kModeResidual = 2 };
 struct __align__(64) ReqInfo {
-    int64_t t_off;   // element offset of the target row pass 2 reads
+    int64_t t_off;   // element offset of the target row of the final draw
     int64_t d_off;   // element offset of the draft row (residual only)
-    double u;        // uniform of the final sample
-    double inv_sp;   // 1 / sum_v exp((l_v - m_t) / T), fp64 (residual only)
-    double inv_sq;   // 1 / sum_v exp((d_v - m_d) / T), fp64 (residual only)
+    double u;        // uniform of the final draw
+    double rho_lo;   // bounds on S_t / S_d (row normalisers relative to their
+    double rho_hi;   //   maxima) from the fp32 pass (residual only)
     float mt, md;    // row maxima
     int mode;        // kMode*
-    int out_index;   // flat index into out_tokens of the sampled token
+    int out_index;   // flat index into out_tokens of the drawn token
 };
 
 enum : int { kLinear = 0, kTreeStochastic = 1, kTreeGreedy = 2 };
+
+// Global work counters of one call (zeroed by the host before the launch).
+struct Counters {
+    unsigned a_next;     // next pass-1 item to claim
+    unsigned p_head;     // next pass-2 item to claim
+    unsigned frontier;   // requests [0, frontier) are decided
+    unsigned finalized;  // requests whose outputs are complete
+};
 
 struct Params {
     const void *tl;          // target logits
@@ -263,11 +360,17 @@ struct Params {
     const int32_t *tokens;   // linear: draft tokens [B][k]; tree: node tokens [B][N]
     const int32_t *parents;  // tree only
     int B, k, N, max_depth, V;
-    int R;                   // rows per request handled by pass 1
+    int R;                   // rows per request streamed by pass 1
     int S;                   // pass-1 segments per row
     int seg;                 // pass-1 segment length (entries)
     int S2;                  // pass-2 segments per row
+    int W32;                 // 32-bit words of one request's ambiguity bitmap
+    unsigned nA, nP;         // pass-1 and pass-2 item counts
+    FastDiv div_req;         // by R * S (pass-1 items per request)
+    FastDiv div_s;           // by S
+    FastDiv div_s2;          // by S2
     float c;                 // log2(e) / T, fp32
+    double c64;              // log2(e) / T, fp64
     double inv_t;            // 1 / T, fp64
     uint64_t seed;
     uint32_t offset;
@@ -276,39 +379,24 @@ struct Params {
     int32_t *path;           // tree only, nullable
     float *dbg_lp, *dbg_lq;  // linear only, nullable
     int32_t *status;         // nullable
-    // workspace regions
-    float2 *rowpart;         // [B][R][S]
-    RowStat *rowstat;        // [B][R]
+    // workspace
+    Counters *ctr;
+    unsigned *a_done, *p2_done, *decided;  // [B] each (a_done counts merged rows)
+    unsigned *row_done;      // [B][R] pass-1 items completed per row
+    float2 *rowpart;         // [B][R][S] pass-1 partials
+    RowStat *rowstat;        // [B][R] merged rows
     ReqInfo *req;            // [B]
-    double2 *p2a;            // [B][S2]
-    double *p2b;             // [B][S2]
-    unsigned *cnt1, *cnt2a, *cnt2b;  // [B] each
+    double4 *p2part;         // [B][S2] (sum e, sum f, sum e over p>q, sum f over p>q)
+    int *p2amb;              // [B][S2] undecided entries per segment
+    unsigned *ambbits;       // [B][W32] undecided entries, one bit each
+    double *p2w;             // [B][S2] final segment weights
+    double2 *p2lane;         // [B][S2][32] per-lane partials of pass 2
+    double exp2tab[64];      // 2^(j/64), j = 0..63
 };
 
 __device__ __forceinline__ void report(int32_t *status, int bits)
 {
     if (status && bits) atomicOr(status, bits);
-}
-
-// "Last block done" counter: returns true in every thread of exactly one
-// block (the last of `total` arrivals); that block resets the counter to
-// zero, so the workspace is left zero-filled for the next call.  Callers
-// write their partial results before calling.  No block ever waits.
-__device__ __forceinline__ bool arrive_last(unsigned *counter, unsigned total)
-{
-    __shared__ int last;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        unsigned prev = atomicAdd(counter, 1u);
-        last = (prev == total - 1);
-        if (last) {
-            atomicExch(counter, 0u);
-            __threadfence();
-        }
-    }
-    __syncthreads();
-    return last != 0;
 }
 
 }  // namespace sv

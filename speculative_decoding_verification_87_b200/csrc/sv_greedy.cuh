@@ -17,7 +17,7 @@
 #include <cooperative_groups.h>
 
 #include "sv_common.cuh"
-#include "sv_stats.cuh"
+
 
 namespace sv {
 
