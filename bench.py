@@ -217,11 +217,13 @@ class Runner:
             self.parents = dev(w.parents)
             W = w.max_depth + 1
             self.out = torch.empty((w.batch, W), dtype=torch.int32, device=device)
-            self.kernels_per_call = 1
+            # pass 1 + decide, then pass 2 + finalize for the stochastic draw
+            self.kernels_per_call = 4 if name == "tree-stochastic" else 2
         else:
             self.tokens = dev(w.tokens.astype(np.int32))
             self.out = torch.empty((w.batch, w.k + 1), dtype=torch.int32, device=device)
-            self.kernels_per_call = 1
+            # greedy: one cluster kernel; linear: pass 1, decide, pass 2, finalize
+            self.kernels_per_call = 1 if name == "greedy" else 4
         self.acc = torch.empty((w.batch,), dtype=torch.int32, device=device)
 
     def call(self, offset, target=None, draft=None, tokens=None):

@@ -1,8 +1,9 @@
 // specverify.cu -- C ABI of libspecverify.so (sm_100a) and its launches.
 //
-// spec_verify_linear / spec_verify_tree: one memset of the work counters and
-// one launch of the persistent engine (sv_engine.cuh) on the caller's
-// stream; no host synchronisation.
+// spec_verify_linear / spec_verify_tree: the pass-1 kernel, the decide
+// kernel and, where a token is drawn, the pass-2 and finalize kernels
+// (sv_verify.cuh), each a programmatic dependent of the one before, on the
+// caller's stream; no host synchronisation and no workspace clearing.
 // spec_verify_greedy: one launch of the cluster kernel (sv_greedy.cuh); no
 // workspace.
 #include <algorithm>
@@ -16,7 +17,7 @@
 
 #include "../../include/specverify.h"
 #include "sv_common.cuh"
-#include "sv_engine.cuh"
+#include "sv_verify.cuh"
 #include "sv_exp64.cuh"
 #include "sv_greedy.cuh"
 #include "sv_philox.cuh"
@@ -35,32 +36,31 @@ __global__ void k_debug_uniforms(uint64_t seed, uint32_t offset, uint32_t purpos
 
 __global__ void k_debug_exp2(const double *z, double *out, int n, int kind, Params p)
 {
+    __shared__ double tab[64];
+    if (threadIdx.x < 64) tab[threadIdx.x] = p.exp2tab[threadIdx.x];
+    __syncthreads();
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    Exp2Table tab;
-    tab.lo = p.exp2tab[threadIdx.x & 31];
-    tab.hi = p.exp2tab[(threadIdx.x & 31) + 32];
-    const double zi = i < n ? z[i] : 0.0;
-    const double v = exp2_fp64(zi, tab);  // every lane calls (warp-collective)
-    if (i < n) {
-        if (kind == 1) out[i] = f32_to_f64(ex2_fma(static_cast<float>(zi)));
-        else if (kind == 2) out[i] = f32_to_f64(ex2_approx(static_cast<float>(zi)));
-        else out[i] = v;
-    }
+    if (i >= n) return;
+    const double zi = z[i];
+    if (kind == 1) out[i] = f32_to_f64(ex2_fma(static_cast<float>(zi)));
+    else if (kind == 2) out[i] = f32_to_f64(ex2_approx(static_cast<float>(zi)));
+    else out[i] = exp2_fp64(zi, tab);
 }
 
 // ------------------------------------------------------------ host helpers
 namespace {
 
 constexpr size_t kAlign = 256;
-constexpr int kBatchF32 = 32 * 4 * F32::kVec;  // smallest pass-1 segment (fp32, one warp batch)
+constexpr int kItemMin = Pass1Shape<F32>::kItem;  // the shorter pass-1 item (fp32)
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-// Workspace layout; the counters (cleared per call) come first.  Region
-// sizes use the smallest pass-1 segment, so any per-call choice fits.
+// Workspace layout.  Every region a call reads is written earlier in the
+// same call, so the workspace needs no clearing.  Region sizes use the
+// shorter pass-1 item, so both dtypes fit.
 struct Layout {
-    size_t ctr, rowpart, rowstat, req, p2part, p2amb, ambbits, p2w, p2lane, total, clear_bytes;
+    size_t rowpart, req, p2part, p2amb, ambbits, p2w, p2lane, total;
     bool ok;
 };
 
@@ -69,17 +69,12 @@ Layout layout(int B, int R, int V)
     Layout L{};
     L.ok = false;
     if (B < 0 || R < 1 || V < 1) return L;
-    const int64_t smax = ceil_div(V, kBatchF32);
+    const int64_t smax = ceil_div(V, kItemMin);
     const int64_t s2 = ceil_div(V, kSeg2);
-    const int64_t w32 = ceil_div(V, 32);
+    const int64_t w32 = s2 * (kSeg2 / 32);  // whole segments (16-byte aligned rows of the bitmap)
     size_t off = 0;
-    L.ctr = off;
-    L.clear_bytes = sizeof(Counters) + sizeof(unsigned) * (3 + static_cast<size_t>(R)) * static_cast<size_t>(B);
-    off = align_up(off + L.clear_bytes);
     L.rowpart = off;
     off = align_up(off + sizeof(float2) * static_cast<size_t>(B) * R * smax);
-    L.rowstat = off;
-    off = align_up(off + sizeof(RowStat) * static_cast<size_t>(B) * R);
     L.req = off;
     off = align_up(off + sizeof(ReqInfo) * static_cast<size_t>(B));
     L.p2part = off;
@@ -100,7 +95,6 @@ Layout layout(int B, int R, int V)
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int elem_size(spec_dtype_t d) { return d == SPEC_BF16 ? 2 : 4; }
-int vec_of(spec_dtype_t d) { return d == SPEC_BF16 ? Bf16::kVec : F32::kVec; }
 
 // Shape checks that hold for every batch size (an empty batch included).
 int check_shape(spec_dtype_t dtype, int64_t stride, int V)
@@ -122,14 +116,7 @@ int check_rows(const void *tl, const void *dl, bool need_dl)
 void fill_workspace(Params &p, void *ws, const Layout &L)
 {
     char *w = static_cast<char *>(ws);
-    p.ctr = reinterpret_cast<Counters *>(w + L.ctr);
-    auto *per_req = reinterpret_cast<unsigned *>(w + L.ctr + sizeof(Counters));
-    p.a_done = per_req;
-    p.p2_done = per_req + p.B;
-    p.decided = per_req + 2 * static_cast<int64_t>(p.B);
-    p.row_done = per_req + 3 * static_cast<int64_t>(p.B);
     p.rowpart = reinterpret_cast<float2 *>(w + L.rowpart);
-    p.rowstat = reinterpret_cast<RowStat *>(w + L.rowstat);
     p.req = reinterpret_cast<ReqInfo *>(w + L.req);
     p.p2part = reinterpret_cast<double4 *>(w + L.p2part);
     p.p2amb = reinterpret_cast<int *>(w + L.p2amb);
@@ -144,35 +131,39 @@ void fill_exp2_table(Params &p)
     for (int j = 0; j < 64; ++j) p.exp2tab[j] = std::exp2(static_cast<double>(j) / 64.0);
 }
 
-// Pass-1 segment: the largest of 4, 2, 1 warp batches that still gives
-// every worker several items.
-int choose_seg(int B, int R, int V, spec_dtype_t dtype, int64_t min_items)
-{
-    const int batch = 32 * 4 * vec_of(dtype);
-    for (int nb : {4, 2}) {
-        const int64_t S = ceil_div(V, static_cast<int64_t>(batch) * nb);
-        if (static_cast<int64_t>(B) * R * S >= min_items) return batch * nb;
-    }
-    return batch;
-}
 
-// Engine occupancy per device and instantiation.
+// Occupancy per device, dtype and mode, of the pass kernels.
 std::mutex g_mu;
-int g_engine_blocks[64][2][3];
+int g_pass1_blocks[64][2][3];
+int g_pass2_blocks[64][2][3];
+bool g_final_attr[64][2][3];
 int g_sm_count[64];
 
-template <class Tag, int MODE>
-int engine_blocks_per_sm(int dev, int dtype_index)
+// Decide dynamic shared memory: the merged statistics of a request's rows.
+size_t decide_smem(int R) { return (sizeof(double) + sizeof(float) + sizeof(int)) * static_cast<size_t>(R); }
+
+// Finalize dynamic shared memory: the segment weights of each warp, for
+// vocabularies up to kMaxS2Shared segments (else the workspace holds them).
+size_t finalize_smem(int S2)
 {
-    int &slot = g_engine_blocks[dev][dtype_index][MODE];
+    return S2 <= kMaxS2Shared ? sizeof(double) * kWarps * static_cast<size_t>(S2) : 0;
+}
+
+template <class Tag, int MODE>
+constexpr int pass1_min_blocks()
+{
+    return 2;
+}
+
+template <class Kernel>
+int blocks_per_sm(int &slot, Kernel kernel, size_t dyn_smem)
+{
     if (slot > 0) return slot;
-    if (cudaFuncSetAttribute(k_engine<Tag, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kRingBytes)) != cudaSuccess)
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(dyn_smem)) != cudaSuccess)
         return -1;
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_engine<Tag, MODE>, kThreads, kRingBytes) !=
-            cudaSuccess ||
-        n < 1)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kThreads, dyn_smem) != cudaSuccess || n < 1)
         return -1;
     slot = n;
     return n;
@@ -189,24 +180,68 @@ int sm_count(int dev)
     return n;
 }
 
-// Clear the counters and launch the engine.
+// A launch that may begin while the previous kernel on the stream drains
+// (the kernel itself waits for it with griddepcontrol.wait).
+template <class Kernel>
+int launch_dependent(Kernel kernel, int64_t blocks, size_t dyn, cudaStream_t st, const Params &p,
+                     int threads = kThreads)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = dyn;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, p) == cudaSuccess ? SPEC_OK : SPEC_ECUDA;
+}
+
+// Launch pass 1, then the decide step and, where a token is drawn, pass 2
+// and the finalize step, each a programmatic dependent of the one before.
+// Pass grids are at most one resident wave.
 template <class Tag, int MODE>
-int launch_engine(Params &p, const Layout &L, void *ws, int dtype_index, cudaStream_t st)
+int launch_verify(Params &p, const Layout &L, void *ws, int dtype_index, cudaStream_t st)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SPEC_ECUDA;
-    int per_sm, sms;
+    constexpr int kMin1 = pass1_min_blocks<Tag, MODE>();
+    const size_t dyn3 = finalize_smem(p.S2);
+    int per_sm1, per_sm2 = 1, sms;
     {
         std::lock_guard<std::mutex> lock(g_mu);
-        per_sm = engine_blocks_per_sm<Tag, MODE>(dev, dtype_index);
+        per_sm1 = blocks_per_sm(g_pass1_blocks[dev][dtype_index][MODE], k_pass1<Tag, MODE, kMin1>, kRingBytes);
+        if (p.nP > 0) {
+            per_sm2 = blocks_per_sm(g_pass2_blocks[dev][dtype_index][MODE], k_pass2<Tag, MODE>,
+                                    StageShape<Tag>::kBytes);
+            bool &attr = g_final_attr[dev][dtype_index][MODE];
+            if (!attr) {
+                if (cudaFuncSetAttribute(k_finalize<Tag, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(finalize_smem(kMaxS2Shared))) != cudaSuccess)
+                    return SPEC_ECUDA;
+                attr = true;
+            }
+        }
         sms = sm_count(dev);
     }
-    if (per_sm < 1 || sms < 1) return SPEC_ECUDA;
-    const int64_t want = ceil_div(static_cast<int64_t>(p.nA) + p.nP, kWarps - kP2Warps);
-    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(static_cast<int64_t>(per_sm) * sms, want));
-    if (cudaMemsetAsync(ws, 0, L.clear_bytes, st) != cudaSuccess) return SPEC_ECUDA;
-    k_engine<Tag, MODE><<<static_cast<unsigned>(blocks), kThreads, kRingBytes, st>>>(p);
-    return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ECUDA;
+    if (per_sm1 < 1 || per_sm2 < 1 || sms < 1) return SPEC_ECUDA;
+    const int64_t blocks1 =
+        std::max<int64_t>(1, std::min<int64_t>(static_cast<int64_t>(per_sm1) * sms, ceil_div(p.nA, kWarps)));
+    k_pass1<Tag, MODE, kMin1><<<static_cast<unsigned>(blocks1), kThreads, kRingBytes, st>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return SPEC_ECUDA;
+    const int64_t blocksd = std::max<int64_t>(1, std::min<int64_t>(static_cast<int64_t>(2) * sms, p.B));
+    if (launch_dependent(k_decide<Tag, MODE>, blocksd, decide_smem(p.R), st, p, kDecideThreads) != SPEC_OK)
+        return SPEC_ECUDA;
+    if (p.nP == 0) return SPEC_OK;
+
+    const int64_t blocks2 =
+        std::max<int64_t>(1, std::min<int64_t>(static_cast<int64_t>(per_sm2) * sms, ceil_div(p.nP, kWarps)));
+    if (launch_dependent(k_pass2<Tag, MODE>, blocks2, StageShape<Tag>::kBytes, st, p) != SPEC_OK)
+        return SPEC_ECUDA;
+    const int64_t blocks3 = std::max<int64_t>(1, std::min<int64_t>(sms, ceil_div(p.B, kWarps)));
+    return launch_dependent(k_finalize<Tag, MODE>, blocks3, dyn3, st, p);
 }
 
 // Largest number of co-resident greedy clusters, per device and dtype.
@@ -281,16 +316,15 @@ void base_params(Params &p, const void *tl, const void *dl, int64_t stride, int 
     p.seed = seed;
     p.offset = offset;
     p.S2 = static_cast<int>(ceil_div(V, kSeg2));
-    p.W32 = static_cast<int>(ceil_div(V, 32));
+    p.W32 = p.S2 * (kSeg2 / 32);
     fill_exp2_table(p);
 }
 
-// Items per request and segment choice shared by the linear and tree calls.
+// Item counts shared by the linear and tree calls.
 int setup_items(Params &p, int R, spec_dtype_t dtype, bool pass2)
 {
     p.R = R;
-    p.seg = choose_seg(p.B, R, p.V, dtype, 16384);
-    p.S = static_cast<int>(ceil_div(p.V, p.seg));
+    p.S = static_cast<int>(ceil_div(p.V, dtype == SPEC_BF16 ? Pass1Shape<Bf16>::kItem : Pass1Shape<F32>::kItem));
     const int64_t nA = static_cast<int64_t>(p.B) * R * p.S;
     const int64_t nP = pass2 ? static_cast<int64_t>(p.B) * p.S2 : 0;
     if (nA >= (int64_t(1) << 31) || nP >= (int64_t(1) << 31)) return SPEC_EUNSUPPORTED;
@@ -363,8 +397,8 @@ extern "C" int spec_verify_linear(const void *target_logits, const void *draft_l
     rc = setup_items(p, R, dtype, true);
     if (rc != SPEC_OK) return rc;
     fill_workspace(p, workspace, L);
-    return dtype == SPEC_BF16 ? launch_engine<Bf16, kLinear>(p, L, workspace, 1, stream)
-                              : launch_engine<F32, kLinear>(p, L, workspace, 0, stream);
+    return dtype == SPEC_BF16 ? launch_verify<Bf16, kLinear>(p, L, workspace, 1, stream)
+                              : launch_verify<F32, kLinear>(p, L, workspace, 0, stream);
 }
 
 extern "C" int spec_verify_greedy(const void *target_logits, spec_dtype_t dtype,
@@ -431,10 +465,10 @@ extern "C" int spec_verify_tree(const void *target_logits, const void *draft_log
     if (rc != SPEC_OK) return rc;
     fill_workspace(p, workspace, L);
     if (dtype == SPEC_BF16)
-        return stochastic ? launch_engine<Bf16, kTreeStochastic>(p, L, workspace, 1, stream)
-                          : launch_engine<Bf16, kTreeGreedy>(p, L, workspace, 1, stream);
-    return stochastic ? launch_engine<F32, kTreeStochastic>(p, L, workspace, 0, stream)
-                      : launch_engine<F32, kTreeGreedy>(p, L, workspace, 0, stream);
+        return stochastic ? launch_verify<Bf16, kTreeStochastic>(p, L, workspace, 1, stream)
+                          : launch_verify<Bf16, kTreeGreedy>(p, L, workspace, 1, stream);
+    return stochastic ? launch_verify<F32, kTreeStochastic>(p, L, workspace, 0, stream)
+                      : launch_verify<F32, kTreeGreedy>(p, L, workspace, 0, stream);
 }
 
 extern "C" int spec_verify_debug_uniforms(uint64_t seed, uint32_t offset, uint32_t purpose,

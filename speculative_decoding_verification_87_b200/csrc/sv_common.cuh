@@ -15,13 +15,13 @@ constexpr int kWarps = kThreads / 32;
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
 // Per-request status bits (mirror SPEC_STATUS_* in the public header).
-enum : int { kStToken = 1, kStTree = 2, kStLogit = 4, kStTimeout = 8 };
+enum : int { kStToken = 1, kStTree = 2, kStLogit = 4 };
 
 // Philox counter purposes.
 enum : uint32_t { kPurposeAccept = 0, kPurposeSample = 1 };
 
 // Pass-2 segment: 2048 vocabulary entries, 64 contiguous entries per lane.
-constexpr int kSeg2 = 2048;
+constexpr int kSeg2 = 512;
 constexpr int kLane2 = kSeg2 / 32;
 
 // Storage tags: element type and entries per 16-byte vector.
@@ -323,13 +323,6 @@ __device__ __forceinline__ int block_max(int v, int *red)
 }
 
 // ------------------------------------------------------- per-call parameters
-// Merged statistics of one logit row.
-struct RowStat {
-    float m;   // row maximum (greedy: maximum value)
-    int idx;   // greedy: argmax (lowest index on ties)
-    double s;  // stochastic: sum_v exp((l_v - m) / T)
-};
-
 // What the final draw of one request needs.
 enum : int { kModeNone = 0, kModeTargetRow = 1, kModeResidual = 2 };
 struct __align__(64) ReqInfo {
@@ -341,17 +334,13 @@ struct __align__(64) ReqInfo {
     float mt, md;    // row maxima
     int mode;        // kMode*
     int out_index;   // flat index into out_tokens of the drawn token
+    float kc;        // (mt - md) c + log2(rho0), rho0 the pass-1 estimate of
+                     //   S_t / S_d: log2(e/f) - log2(rho0) = (l_t - l_d) c - kc
+    float tcls;      // |(l_t - l_d) c - kc| <= tcls: the sign of p - q is not
+                     //   certain from fp32 (residual only)
 };
 
 enum : int { kLinear = 0, kTreeStochastic = 1, kTreeGreedy = 2 };
-
-// Global work counters of one call (zeroed by the host before the launch).
-struct Counters {
-    unsigned a_next;     // next pass-1 item to claim
-    unsigned p_head;     // next pass-2 item to claim
-    unsigned frontier;   // requests [0, frontier) are decided
-    unsigned finalized;  // requests whose outputs are complete
-};
 
 struct Params {
     const void *tl;          // target logits
@@ -361,8 +350,7 @@ struct Params {
     const int32_t *parents;  // tree only
     int B, k, N, max_depth, V;
     int R;                   // rows per request streamed by pass 1
-    int S;                   // pass-1 segments per row
-    int seg;                 // pass-1 segment length (entries)
+    int S;                   // pass-1 items per row
     int S2;                  // pass-2 segments per row
     int W32;                 // 32-bit words of one request's ambiguity bitmap
     unsigned nA, nP;         // pass-1 and pass-2 item counts
@@ -380,11 +368,7 @@ struct Params {
     float *dbg_lp, *dbg_lq;  // linear only, nullable
     int32_t *status;         // nullable
     // workspace
-    Counters *ctr;
-    unsigned *a_done, *p2_done, *decided;  // [B] each (a_done counts merged rows)
-    unsigned *row_done;      // [B][R] pass-1 items completed per row
     float2 *rowpart;         // [B][R][S] pass-1 partials
-    RowStat *rowstat;        // [B][R] merged rows
     ReqInfo *req;            // [B]
     double4 *p2part;         // [B][S2] (sum e, sum f, sum e over p>q, sum f over p>q)
     int *p2amb;              // [B][S2] undecided entries per segment

@@ -4,12 +4,13 @@
 // function in IEEE floating-point arithmetic", ACM TOMS 15(2), 1989.
 // Reduce z = e + j/64 + r with integer e, j in [0, 64) and |r| <= 1/128;
 // 2^z = 2^e * 2^(j/64) * 2^r, where 2^(j/64) comes from a 64-entry table and
-// 2^r = exp(r ln 2) from its Taylor polynomial of degree 5 (the first omitted
-// term is below (ln2/128)^6 / 720 ~ 3.5e-17 relative).
+// 2^r = 1 + r q(r) with q(r) = (2^r - 1)/r from the Taylor series of
+// exp(r ln 2) (the first omitted term is below (ln2/128)^6 / 720 ~ 3.5e-17
+// relative).  2^(j/64 + r) is formed as tj + (tj r) q(r), so the product
+// tj r runs beside the Horner chain.
 //
-// The table lives in registers, two entries per lane (lane L holds
-// 2^(L/64) and 2^((L+32)/64)), and is read with a warp shuffle, so every
-// lane of the warp must call exp2_fp64 together.
+// The table (2^(j/64), j = 0..63, 512 bytes) lives in shared memory; the
+// caller fills it once per block.
 #pragma once
 
 #include <cstdint>
@@ -24,35 +25,25 @@ constexpr double kE3 = kE2 * kLn2 / 3.0;
 constexpr double kE4 = kE3 * kLn2 / 4.0;
 constexpr double kE5 = kE4 * kLn2 / 5.0;
 
-// Two table entries of this lane: 2^(lane/64) (lo) and 2^((lane+32)/64) (hi).
-struct Exp2Table {
-    double lo, hi;
-};
-
-// 2^z for z <= 0.  Results below 2^-1020 are returned as 0 (they cannot
-// move a sum whose largest term is 1).  Warp-collective.
-__device__ __forceinline__ double exp2_fp64(double z, const Exp2Table &tab)
+// 2^z for z <= 0.  Results below 2^-1020 (and NaN arguments) give 0: such
+// terms cannot move a sum whose largest term is 1, and an entry whose logit
+// is -inf must keep weight exactly 0.  2^floor(k/64) enters the exponent
+// field of the table value, beside the polynomial chain.
+__device__ __forceinline__ double exp2_fp64(double z, const double *tab)
 {
-    const bool tiny = !(z > -1020.0);
-    const double zz = tiny ? 0.0 : z;
     constexpr double kMagic = 6755399441055744.0;  // 1.5 * 2^52: rounds to an integer
-    const double t = fma(zz, 64.0, kMagic);
-    const int k = __double2loint(t);               // round(64 z), two's complement
-    const double kd = t - kMagic;
-    const double r = fma(kd, -0.015625, zz);       // z - k/64, exact
-    double p = fma(kE5, r, kE4);
-    p = fma(p, r, kE3);
-    p = fma(p, r, kE2);
-    p = fma(p, r, kE1);
-    p = p * r;                                     // 2^r - 1
-    const int j = k & 63;
-    const double lo = __shfl_sync(0xFFFFFFFFu, tab.lo, j & 31);
-    const double hi = __shfl_sync(0xFFFFFFFFu, tab.hi, j & 31);
-    const double tj = (j & 32) ? hi : lo;          // 2^(j/64)
-    const double y = fma(tj, p, tj);               // 2^(j/64 + r), in [1, 2)
-    const int e = k >> 6;                          // floor(k / 64), >= -1020
-    const double scaled = __hiloint2double(__double2hiint(y) + (e << 20), __double2loint(y));
-    return tiny ? 0.0 : scaled;
+    const double t = fma(z, 64.0, kMagic);
+    const int k = __double2loint(t);                    // round(64 z), two's complement
+    const double r = fma(t - kMagic, -0.015625, z);     // z - k/64, exact
+    const double tj = tab[k & 63];                      // 2^(j/64)
+    const unsigned ehi = static_cast<unsigned>(__double2hiint(tj)) + (static_cast<unsigned>(k >> 6) << 20);
+    const double ts = __hiloint2double(static_cast<int>(ehi), __double2loint(tj));  // 2^(k/64), for z > -1020
+    double q = fma(kE5, r, kE4);
+    q = fma(q, r, kE3);
+    q = fma(q, r, kE2);
+    q = fma(q, r, kE1);
+    const double y = fma(ts * r, q, ts);
+    return z > -1020.0 ? y : 0.0;
 }
 
 // Exact widening of a bf16 bit pattern (low 16 bits of h) to fp64 with
