@@ -60,7 +60,7 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // same call, so the workspace needs no clearing.  Region sizes use the
 // shorter pass-1 item, so both dtypes fit.
 struct Layout {
-    size_t rowpart, req, p2part, p2amb, ambbits, p2w, p2lane, total;
+    size_t rowpart, req, p2part, p2amb, ambbits, p2w, total;
     bool ok;
 };
 
@@ -84,9 +84,7 @@ Layout layout(int B, int R, int V)
     L.ambbits = off;
     off = align_up(off + sizeof(unsigned) * static_cast<size_t>(B) * w32);
     L.p2w = off;
-    off = align_up(off + sizeof(double) * static_cast<size_t>(B) * s2);
-    L.p2lane = off;
-    off = align_up(off + sizeof(double2) * 32 * static_cast<size_t>(B) * s2);
+    off = align_up(off + 2 * sizeof(double) * static_cast<size_t>(B) * s2);
     L.total = off < kAlign ? kAlign : off;
     L.ok = true;
     return L;
@@ -122,7 +120,6 @@ void fill_workspace(Params &p, void *ws, const Layout &L)
     p.p2amb = reinterpret_cast<int *>(w + L.p2amb);
     p.ambbits = reinterpret_cast<unsigned *>(w + L.ambbits);
     p.p2w = reinterpret_cast<double *>(w + L.p2w);
-    p.p2lane = reinterpret_cast<double2 *>(w + L.p2lane);
 }
 
 // 2^(j/64), j = 0..63, from the host math library.
@@ -146,7 +143,7 @@ size_t decide_smem(int R) { return (sizeof(double) + sizeof(float) + sizeof(int)
 // vocabularies up to kMaxS2Shared segments (else the workspace holds them).
 size_t finalize_smem(int S2)
 {
-    return S2 <= kMaxS2Shared ? sizeof(double) * kWarps * static_cast<size_t>(S2) : 0;
+    return S2 <= kMaxS2Shared ? 2 * sizeof(double) * kWarps * static_cast<size_t>(S2) : 0;
 }
 
 template <class Tag, int MODE>

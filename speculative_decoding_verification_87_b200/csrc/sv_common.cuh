@@ -373,8 +373,7 @@ struct Params {
     double4 *p2part;         // [B][S2] (sum e, sum f, sum e over p>q, sum f over p>q)
     int *p2amb;              // [B][S2] undecided entries per segment
     unsigned *ambbits;       // [B][W32] undecided entries, one bit each
-    double *p2w;             // [B][S2] final segment weights
-    double2 *p2lane;         // [B][S2][32] per-lane partials of pass 2
+    double *p2w;             // [B][2][S2] finalize scratch (vocabularies too large for shared memory)
     double exp2tab[64];      // 2^(j/64), j = 0..63
 };
 

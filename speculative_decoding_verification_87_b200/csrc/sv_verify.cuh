@@ -236,49 +236,22 @@ __device__ __forceinline__ void issue_item(const Item1 &it, uint4 *slot)
     constexpr int kEsz = sizeof(typename Tag::elem);
     const int lane = threadIdx.x & 31;
     if (!it.active) return;
+    const char *src = it.row + static_cast<int64_t>(it.e_begin + lane * kVec) * kEsz;
+    const unsigned dst = static_cast<unsigned>(__cvta_generic_to_shared(slot + lane));
+    if (it.e_begin + Pass1Shape<Tag>::kItem <= it.e_end) {
+#pragma unroll
+        for (int v = 0; v < Pass1Shape<Tag>::kVecL; ++v)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst + v * 512),
+                         "l"(src + v * 32 * kVec * kEsz) : "memory");
+        return;
+    }
 #pragma unroll
     for (int v = 0; v < Pass1Shape<Tag>::kVecL; ++v) {
         const int e0 = it.e_begin + (v * 32 + lane) * kVec;
-        if (e0 < it.e_end) {
-            const char *src = it.row + static_cast<int64_t>(e0) * kEsz;
-            const unsigned dst = static_cast<unsigned>(__cvta_generic_to_shared(slot + v * 32 + lane));
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
-        }
+        if (e0 < it.e_end)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst + v * 512),
+                         "l"(src + v * 32 * kVec * kEsz) : "memory");
     }
-}
-
-// Two fp32 values in one 64-bit register pair, for the packed fp32x2 FMA
-// of sm_100.
-typedef unsigned long long f32x2;
-__device__ __forceinline__ f32x2 f2_pack(uint32_t lo, uint32_t hi)
-{
-    f32x2 r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
-    return r;
-}
-__device__ __forceinline__ void f2_unpack(f32x2 v, float &lo, float &hi)
-{
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ f32x2 f2_fma(f32x2 a, f32x2 b, f32x2 c)
-{
-    f32x2 r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-    return r;
-}
-
-// The fp32 bit patterns of the two entries of one 32-bit word of a vector.
-template <class Tag>
-__device__ __forceinline__ f32x2 word_pair(uint32_t w0, uint32_t w1);
-template <>
-__device__ __forceinline__ f32x2 word_pair<Bf16>(uint32_t w, uint32_t)
-{
-    return f2_pack(w << 16, w & 0xFFFF0000u);
-}
-template <>
-__device__ __forceinline__ f32x2 word_pair<F32>(uint32_t w0, uint32_t w1)
-{
-    return f2_pack(w0, w1);
 }
 
 // NaN-propagating max of this lane's vectors of an item.
@@ -318,10 +291,9 @@ __device__ __forceinline__ float lane_max<F32>(const uint4 (&raw)[Pass1Shape<F32
 }
 
 // Reduce one staged item and store its partial.  Stochastic: each lane
-// takes its own max m, then sums 2^(x c - fl(m c)): the exponents of two
-// entries by one packed fp32x2 FMA, one special-function exponential per
-// entry, four independent sums; the lane sums are corrected for
-// fl(m c) - m c and rescaled to the warp max.
+// takes its own max m, then sums 2^(x c - fl(m c)): one FMA and one
+// special-function exponential per entry, four independent sums; the lane
+// sums are corrected for fl(m c) - m c and rescaled to the warp max.
 template <class Tag, int MODE>
 __device__ __forceinline__ void reduce_item1(const Params &p, const Item1 &it, const uint4 *slot)
 {
@@ -373,20 +345,14 @@ __device__ __forceinline__ void reduce_item1(const Params &p, const Item1 &it, c
         const float c = p.c;
         const float m = lane_max<Tag>(raw);
         const float mc = (m == -INFINITY) ? 0.f : m * c;  // all -inf: every term is 0
-        const f32x2 c2 = f2_pack(__float_as_uint(c), __float_as_uint(c));
-        const f32x2 n2 = f2_pack(__float_as_uint(-mc), __float_as_uint(-mc));
+        const float nmc = -mc;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int v = 0; v < kV; ++v) {
-            const uint32_t w[4] = {raw[v].x, raw[v].y, raw[v].z, raw[v].w};
+            float x[kVec];
+            unpack<Tag>(raw[v], x);
 #pragma unroll
-            for (int i = 0; i < 4; i += (kVec == 8 ? 1 : 2)) {
-                const f32x2 z = f2_fma(word_pair<Tag>(w[i], w[(i + 1) & 3]), c2, n2);
-                float z0, z1;
-                f2_unpack(z, z0, z1);
-                acc[i & 3] += ex2_approx(z0);
-                acc[(i + 1) & 3] += ex2_approx(z1);
-            }
+            for (int e = 0; e < kVec; ++e) acc[e & 3] += ex2_approx(fmaf(x[e], c, nmc));
         }
         const float lsum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
         const float M = warp_max_nan(m);
@@ -508,8 +474,32 @@ __device__ __forceinline__ void merge_row(const Params &p, int b, int r, RowStat
 }
 
 // ------------------------------------------------------------------ decide
+// Lane j < k of warp 0 has read the draft token x_j and the target and
+// draft logits at x_j (inputs, so read before pass 1 completes).
+struct DraftProbe {
+    int x;
+    float lt, ld;
+};
+
 template <class Tag>
-__device__ __forceinline__ void decide_linear(const Params &p, int b, RowStats sh)
+__device__ __forceinline__ DraftProbe probe_drafts(const Params &p, int b)
+{
+    const int lane = threadIdx.x & 31;
+    DraftProbe d;
+    d.x = -1;
+    d.lt = d.ld = 0.f;
+    if (b < p.B && lane < p.k) {
+        d.x = __ldg(p.tokens + static_cast<int64_t>(b) * p.k + lane);
+        if (d.x >= 0 && d.x < p.V) {
+            d.lt = load_logit<Tag>(p.tl, (static_cast<int64_t>(b) * (p.k + 1) + lane) * p.stride + d.x);
+            d.ld = load_logit<Tag>(p.dl, (static_cast<int64_t>(b) * p.k + lane) * p.stride + d.x);
+        }
+    }
+    return d;
+}
+
+template <class Tag>
+__device__ __forceinline__ void decide_linear(const Params &p, int b, RowStats sh, const DraftProbe &pr)
 {
     const int lane = threadIdx.x & 31;
     const int k = p.k, R = p.R;
@@ -520,7 +510,7 @@ __device__ __forceinline__ void decide_linear(const Params &p, int b, RowStats s
     int x = -1;
     bool tok_ok = true;
     if (lane < k) {
-        x = __ldg(p.tokens + static_cast<int64_t>(b) * k + lane);
+        x = pr.x;
         tok_ok = (x >= 0 && x < p.V);
     }
     const bool tok_bad = __any_sync(kFull, !tok_ok);
@@ -529,8 +519,8 @@ __device__ __forceinline__ void decide_linear(const Params &p, int b, RowStats s
     bool acc = true;
     float lpf = __int_as_float(0x7FC00000), lqf = lpf;
     if (lane < k && !bits) {
-        const double lt = logit_f64_at<Tag>(p.tl, (static_cast<int64_t>(b) * (k + 1) + lane) * p.stride + x);
-        const double ld = logit_f64_at<Tag>(p.dl, (static_cast<int64_t>(b) * k + lane) * p.stride + x);
+        const double lt = f32_to_f64(pr.lt);
+        const double ld = f32_to_f64(pr.ld);
         const double lp = (lt - static_cast<double>(sh.m[lane])) * p.inv_t - log(sh.s[lane]);
         const double lq = (ld - static_cast<double>(sh.m[k + 1 + lane])) * p.inv_t - log(sh.s[k + 1 + lane]);
         const double u = philox_uniform(p.seed, static_cast<uint32_t>(b), static_cast<uint32_t>(lane),
@@ -867,6 +857,56 @@ __device__ __forceinline__ double lane_exact_sum(const Params &p, const ReqInfo 
     return w;
 }
 
+// Exact weights of this lane's kLane2 entries [lo, lo + kLane2) into w[],
+// read as whole vectors; returns their sum in index order.
+template <class Tag>
+__device__ __forceinline__ double lane_exact_weights(const Params &p, const ReqInfo &info, bool residual, int lo,
+                                                     double isp, double isq, const double *tab,
+                                                     double (&w)[kLane2])
+{
+    constexpr int kVec = Tag::kVec;
+    constexpr int kEsz = sizeof(typename Tag::elem);
+    constexpr int kNV = kLane2 / kVec;
+    const char *trow = static_cast<const char *>(p.tl) + info.t_off * kEsz;
+    const char *drow = static_cast<const char *>(p.dl) + info.d_off * kEsz;
+    const double nmt = neg_mc(p, info.mt), nmd = neg_mc(p, info.md);
+    uint4 tv[kNV], dv[kNV];
+#pragma unroll
+    for (int v = 0; v < kNV; ++v) {
+        const int e0 = lo + v * kVec;
+        const bool in = e0 < p.V;
+        tv[v] = in ? __ldcg(reinterpret_cast<const uint4 *>(trow + static_cast<int64_t>(e0) * kEsz))
+                   : make_uint4(0, 0, 0, 0);
+        dv[v] = (in && residual) ? __ldcg(reinterpret_cast<const uint4 *>(drow + static_cast<int64_t>(e0) * kEsz))
+                                 : make_uint4(0, 0, 0, 0);
+    }
+    double sum = 0.0;
+#pragma unroll
+    for (int v = 0; v < kNV; ++v) {
+        const int e0 = lo + v * kVec;
+        if (e0 + kVec > p.V) {
+            tv[v] = mask_tail<Tag>(tv[v], p.V - e0);
+            dv[v] = mask_tail<Tag>(dv[v], p.V - e0);
+        }
+        float xt[kVec], xd[kVec];
+        unpack<Tag>(tv[v], xt);
+        unpack<Tag>(dv[v], xd);
+#pragma unroll
+        for (int e = 0; e < kVec; ++e) {
+            const double et = exp2_fp64(entry_z(p, xt[e], nmt), tab);
+            double we = et;
+            if (residual) {
+                const double ef = exp2_fp64(entry_z(p, xd[e], nmd), tab);
+                const double pp = et * isp, qq = ef * isq;
+                we = pp > qq ? pp - qq : 0.0;
+            }
+            w[v * kVec + e] = we;
+            sum += we;
+        }
+    }
+    return sum;
+}
+
 // Exact weights, summed in index order, of the marked entries among the
 // n32 bitmap words starting at word w0 (n32 = 16: a whole segment, read as
 // four 16-byte loads; n32 = 1: one word, keeping the bits of [lo, lo+16)).
@@ -1008,10 +1048,11 @@ __device__ __forceinline__ int icdf_blocked(const double *W, int n, double u, do
 
 // Draw the token of request b by inverse CDF: segment weights (closed form
 // from the decided sums plus the exact weights of the marked entries), then
-// the lane chunk of the chosen segment, then its entries.  One warp; W: S2
-// doubles of scratch.  Global reads are issued kU segments at a time.
+// exact weights of the chosen segment's entries, read once (16 per lane):
+// lane sums pick the chunk, the owning lane walks it.  One warp; W, B: S2
+// doubles of scratch each.  The sums of a segment are read in one round.
 template <class Tag>
-__device__ __forceinline__ void finalize(const Params &p, int b, const double *tab, double *W)
+__device__ __forceinline__ void finalize(const Params &p, int b, const double *tab, double *W, double *B)
 {
     constexpr int kU = 8;
     const int lane = threadIdx.x & 31;
@@ -1020,32 +1061,39 @@ __device__ __forceinline__ void finalize(const Params &p, int b, const double *t
     const double4 *part = p.p2part + static_cast<int64_t>(b) * S2;
     const int *namb = p.p2amb + static_cast<int64_t>(b) * S2;
     const unsigned *bits = p.ambbits + static_cast<int64_t>(b) * p.W32;
-    bool residual = info.mode == kModeResidual;
-    double isp = 1.0, isq = 1.0;
-    bool exact_all = false;
-
-    if (residual) {
-        double Sp = 0.0, Sq = 0.0;
-        for (int s0 = 0; s0 < S2; s0 += 32 * kU) {
-            double2 ef[kU];
+    double Sp = 0.0, Sq = 0.0;
+    unsigned marked = 0u;  // bit j: segment 32 j + lane (mod 1024) holds marked entries
+    for (int s0 = 0; s0 < S2; s0 += 32 * kU) {
+        double4 pv[kU];
+        int na[kU];
 #pragma unroll
-            for (int j = 0; j < kU; ++j) {
-                const int s = s0 + j * 32 + lane;
-                ef[j] = s < S2 ? __ldcg(reinterpret_cast<const double2 *>(part + s)) : make_double2(0.0, 0.0);
-            }
+        for (int j = 0; j < kU; ++j) {
+            const int s = s0 + j * 32 + lane;
+            pv[j] = s < S2 ? ldcg_d4(part + s) : make_double4(0.0, 0.0, 0.0, 0.0);
+            na[j] = s < S2 ? __ldcg(namb + s) : 0;
+        }
 #pragma unroll
-            for (int j = 0; j < kU; ++j) {
-                Sp += ef[j].x;
-                Sq += ef[j].y;
+        for (int j = 0; j < kU; ++j) {
+            const int s = s0 + j * 32 + lane;
+            if (s < S2) {
+                Sp += pv[j].x;
+                Sq += pv[j].y;
+                W[s] = pv[j].z;
+                B[s] = pv[j].w;
+                if (na[j] > 0) marked |= 1u << ((s >> 5) & 31);
             }
         }
+    }
+    bool residual = info.mode == kModeResidual;
+    double isp = 1.0, isq = 1.0;
+    if (residual) {
         Sp = warp_sum(Sp);
         Sq = warp_sum(Sq);
         isp = 1.0 / Sp;
         isq = 1.0 / Sq;
         const double rho = Sp / Sq;
-        exact_all = !(rho >= info.rho_lo && rho <= info.rho_hi);
-        if (exact_all) {
+        __syncwarp();
+        if (!(rho >= info.rho_lo && rho <= info.rho_hi)) {
             // the pass-1 estimate missed: every weight exactly, a segment at a time
             for (int s = 0; s < S2; ++s) {
                 const double w =
@@ -1053,25 +1101,9 @@ __device__ __forceinline__ void finalize(const Params &p, int b, const double *t
                 if (lane == 0) W[s] = w;
             }
         } else {
-            unsigned marked = 0u;  // bit j: segment s0 + 32 j + lane holds marked entries
-            for (int s0 = 0; s0 < S2; s0 += 32 * kU) {
-                double2 ab[kU];
-                int na[kU];
-#pragma unroll
-                for (int j = 0; j < kU; ++j) {
-                    const int s = s0 + j * 32 + lane;
-                    ab[j] = s < S2 ? __ldcg(reinterpret_cast<const double2 *>(part + s) + 1) : make_double2(0.0, 0.0);
-                    na[j] = s < S2 ? __ldcg(namb + s) : 0;
-                }
-#pragma unroll
-                for (int j = 0; j < kU; ++j) {
-                    const int s = s0 + j * 32 + lane;
-                    if (s < S2) {
-                        const double w = ab[j].x * isp - ab[j].y * isq;
-                        W[s] = w > 0.0 ? w : 0.0;
-                        if (na[j] > 0) marked |= 1u << ((s >> 5) & 31);
-                    }
-                }
+            for (int s = lane; s < S2; s += 32) {
+                const double w = W[s] * isp - B[s] * isq;
+                W[s] = w > 0.0 ? w : 0.0;
             }
             // this lane's segments that hold marked entries
             while (marked) {
@@ -1087,12 +1119,9 @@ __device__ __forceinline__ void finalize(const Params &p, int b, const double *t
         for (int s = lane; s < S2; s += 32) z += W[s];
         if (!(warp_sum(z) > 0.0)) {  // residual mass vanished in rounding: draw from target row n
             residual = false;
-            exact_all = true;  // lane sums below are recomputed (p2lane holds residual sums)
             __syncwarp();
             for (int s = lane; s < S2; s += 32) W[s] = ldcg_d4(part + s).x;
         }
-    } else {
-        for (int s = lane; s < S2; s += 32) W[s] = ldcg_d4(part + s).z;
     }
     __syncwarp();
     double before, Z;
@@ -1100,22 +1129,10 @@ __device__ __forceinline__ void finalize(const Params &p, int b, const double *t
     if (sstar < 0) sstar = 0;
     const double tseg = info.u * Z - before;
 
-    // lane chunks of the chosen segment
-    const int clo = sstar * kSeg2 + lane * kLane2;
-    double lane_w;
-    if (exact_all) {
-        lane_w = lane_exact_sum<Tag>(p, info, residual, clo, isp, isq, tab);
-    } else {
-        const double2 pl = __ldcg(p.p2lane + (static_cast<int64_t>(b) * S2 + sstar) * 32 + lane);
-        if (residual) {
-            const double w = pl.x * isp - pl.y * isq;
-            // this lane's 16 entries are one half of bitmap word clo / 32
-            const unsigned keep = (clo & 31) ? 0xFFFF0000u : 0x0000FFFFu;
-            lane_w = (w > 0.0 ? w : 0.0) + marked_sum<Tag, 1>(p, info, bits, clo >> 5, keep, isp, isq, tab);
-        } else {
-            lane_w = pl.x;
-        }
-    }
+    // the chosen segment: exact weights, 16 entries per lane
+    double wl[kLane2];
+    const double lane_w =
+        lane_exact_weights<Tag>(p, info, residual, sstar * kSeg2 + lane * kLane2, isp, isq, tab, wl);
     const double incl = warp_incl_scan(lane_w);
     double excl = __shfl_up_sync(kFull, incl, 1);
     if (lane == 0) excl = 0.0;
@@ -1128,23 +1145,22 @@ __device__ __forceinline__ void finalize(const Params &p, int b, const double *t
         cl = pos ? 31 - __clz(pos) : 0;
     }
     const double tchunk = tseg - __shfl_sync(kFull, excl, cl);
-
-    // entries of chunk cl, one per lane
-    const int idx = sstar * kSeg2 + cl * kLane2 + lane;
-    const bool valid = lane < kLane2 && idx < p.V;
-    const double w1 = valid ? exact_weight<Tag>(p, info, residual, idx, isp, isq, tab) : 0.0;
-    const double pincl = warp_incl_scan(w1);
-    const unsigned ehit = __ballot_sync(kFull, w1 > 0.0 && pincl > tchunk);
-    int token;
-    if (ehit) {
-        token = sstar * kSeg2 + cl * kLane2 + __ffs(ehit) - 1;
-    } else {
-        const unsigned pos = __ballot_sync(kFull, w1 > 0.0);
-        token = pos ? sstar * kSeg2 + cl * kLane2 + 31 - __clz(pos) : sstar * kSeg2 + cl * kLane2;
+    int e_hit = -1, e_last = -1;
+    if (lane == cl) {
+        double run = 0.0;
+#pragma unroll
+        for (int e = 0; e < kLane2; ++e) {
+            run += wl[e];
+            if (wl[e] > 0.0) {
+                e_last = e;
+                if (e_hit < 0 && run > tchunk) e_hit = e;
+            }
+        }
     }
-    if (lane == 0) {
-        p.out[info.out_index] = token;
-    }
+    e_hit = __shfl_sync(kFull, e_hit, cl);
+    e_last = __shfl_sync(kFull, e_last, cl);
+    const int e_tok = e_hit >= 0 ? e_hit : (e_last >= 0 ? e_last : 0);
+    if (lane == 0) p.out[info.out_index] = sstar * kSeg2 + cl * kLane2 + e_tok;
 }
 
 // One pass-2 item: reduce, then publish the sums, the per-lane partials
@@ -1156,7 +1172,6 @@ __device__ __forceinline__ void p2_item(const Params &p, int b, int s2, const It
     const int lane = threadIdx.x & 31;
     const P2Acc a = reduce_item<Tag, kResidual>(p, it, s2, buf, tab);
     const int64_t at = static_cast<int64_t>(b) * p.S2 + s2;
-    __stcg(p.p2lane + at * 32 + lane, make_double2(a.A, a.B));
     int namb = 0;
     if (kResidual) {
         // two lanes' 16-entry masks form one bitmap word
@@ -1206,6 +1221,8 @@ __global__ void __launch_bounds__(kDecideThreads) k_decide(const __grid_constant
     rs.m = reinterpret_cast<float *>(rowmem + p.R);
     rs.idx = reinterpret_cast<int *>(rs.m + p.R);
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+    DraftProbe pr;
+    if (MODE == kLinear && warp == 0) pr = probe_drafts<Tag>(p, blockIdx.x);
     asm volatile("griddepcontrol.wait;\n" ::: "memory");
     for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
         if (MODE != kLinear) {
@@ -1225,8 +1242,12 @@ __global__ void __launch_bounds__(kDecideThreads) k_decide(const __grid_constant
         }
         __syncthreads();
         if (warp == 0) {
-            if constexpr (MODE == kLinear) decide_linear<Tag>(p, b, rs);
-            else decide_tree<Tag, MODE>(p, b, rs, ts);
+            if constexpr (MODE == kLinear) {
+                decide_linear<Tag>(p, b, rs, pr);
+                pr = probe_drafts<Tag>(p, b + gridDim.x);
+            } else {
+                decide_tree<Tag, MODE>(p, b, rs, ts);
+            }
         }
         __syncthreads();
     }
@@ -1235,7 +1256,7 @@ __global__ void __launch_bounds__(kDecideThreads) k_decide(const __grid_constant
 // Pass 2: (request, segment) items, two ahead: while item i is reduced,
 // item i+1 is being copied and the request record of item i+2 is read.
 template <class Tag, int MODE>
-__global__ void __launch_bounds__(kThreads, 2) k_pass2(const __grid_constant__ Params p)
+__global__ void __launch_bounds__(kThreads, 3) k_pass2(const __grid_constant__ Params p)
 {
     extern __shared__ uint4 dyn[];
     __shared__ double tab[64];
@@ -1312,8 +1333,8 @@ __global__ void __launch_bounds__(kThreads) k_finalize(const __grid_constant__ P
     asm volatile("griddepcontrol.wait;\n" ::: "memory");
     for (int b = blockIdx.x * kWarps + warp; b < p.B; b += gridDim.x * kWarps) {
         if (__ldcg(&p.req[b].mode) == kModeNone) continue;
-        double *W = w_shared ? wdyn + warp * p.S2 : p.p2w + static_cast<int64_t>(b) * p.S2;
-        finalize<Tag>(p, b, tab, W);
+        double *W = w_shared ? wdyn + 2 * warp * p.S2 : p.p2w + 2 * static_cast<int64_t>(b) * p.S2;
+        finalize<Tag>(p, b, tab, W, W + p.S2);
     }
 }
 
