@@ -81,8 +81,12 @@ enum {
     SPEC_STATUS_TOKEN = 1,   /* a draft or node token outside [0, V)                     */
     SPEC_STATUS_TREE = 2,    /* parents[0] != -1, parents[i] not in [0, i), or a node
                                 deeper than max_depth                                    */
-    SPEC_STATUS_LOGIT = 4    /* a NaN logit, or a row with no finite normaliser
+    SPEC_STATUS_LOGIT = 4,   /* a NaN logit, or a row with no finite normaliser
                                 (+inf present, or every entry -inf)                      */
+    SPEC_STATUS_TIMEOUT = 8  /* spec_verify_linear: a warp gave up waiting (about a
+                                second) for another step of the same call; requests not
+                                yet complete have undefined outputs.  Only possible when
+                                the kernel's blocks are not all resident at once.       */
 };
 
 /* Limits checked on the host. */

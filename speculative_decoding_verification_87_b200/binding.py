@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libspecverify.so")
 
 SPEC_F32, SPEC_BF16 = 0, 1
 SPEC_OK = 0
-STATUS_TOKEN, STATUS_TREE, STATUS_LOGIT = 1, 2, 4
+STATUS_TOKEN, STATUS_TREE, STATUS_LOGIT, STATUS_TIMEOUT = 1, 2, 4, 8
 MAX_K, MAX_NODES = 32, 1024
 SYMBOLS = ("spec_verify_workspace_size", "spec_verify_strerror", "spec_verify_linear",
            "spec_verify_greedy", "spec_verify_tree", "spec_verify_debug_uniforms",

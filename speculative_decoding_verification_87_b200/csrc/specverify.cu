@@ -18,6 +18,7 @@
 #include "../../include/specverify.h"
 #include "sv_common.cuh"
 #include "sv_verify.cuh"
+#include "sv_fused.cuh"
 #include "sv_exp64.cuh"
 #include "sv_greedy.cuh"
 #include "sv_philox.cuh"
@@ -57,10 +58,11 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Workspace layout.  Every region a call reads is written earlier in the
-// same call, so the workspace needs no clearing.  Region sizes use the
-// shorter pass-1 item, so both dtypes fit.
+// same call; the one-kernel path first sets its counters and the pass-1
+// partials (which follow them) to all ones.  Region sizes use the shorter
+// pass-1 item, so both dtypes fit.
 struct Layout {
-    size_t rowpart, req, p2part, p2amb, ambbits, p2w, total;
+    size_t counters, rowpart, req, p2part, p2amb, ambbits, p2w, p2lane, total;
     bool ok;
 };
 
@@ -73,6 +75,8 @@ Layout layout(int B, int R, int V)
     const int64_t s2 = ceil_div(V, kSeg2);
     const int64_t w32 = s2 * (kSeg2 / 32);  // whole segments (16-byte aligned rows of the bitmap)
     size_t off = 0;
+    L.counters = off;  // p2cnt[B], decided[B], p2claim; rowpart follows directly
+    off = align_up(off + sizeof(unsigned) * (2 * static_cast<size_t>(B) + 1));
     L.rowpart = off;
     off = align_up(off + sizeof(float2) * static_cast<size_t>(B) * R * smax);
     L.req = off;
@@ -85,6 +89,8 @@ Layout layout(int B, int R, int V)
     off = align_up(off + sizeof(unsigned) * static_cast<size_t>(B) * w32);
     L.p2w = off;
     off = align_up(off + 2 * sizeof(double) * static_cast<size_t>(B) * s2);
+    L.p2lane = off;
+    off = align_up(off + sizeof(double2) * 32 * static_cast<size_t>(B) * s2);
     L.total = off < kAlign ? kAlign : off;
     L.ok = true;
     return L;
@@ -114,12 +120,17 @@ int check_rows(const void *tl, const void *dl, bool need_dl)
 void fill_workspace(Params &p, void *ws, const Layout &L)
 {
     char *w = static_cast<char *>(ws);
+    auto *cnt = reinterpret_cast<unsigned *>(w + L.counters);
+    p.p2cnt = cnt;
+    p.decided = cnt + p.B;
+    p.p2claim = p.decided + p.B;
     p.rowpart = reinterpret_cast<float2 *>(w + L.rowpart);
     p.req = reinterpret_cast<ReqInfo *>(w + L.req);
     p.p2part = reinterpret_cast<double4 *>(w + L.p2part);
     p.p2amb = reinterpret_cast<int *>(w + L.p2amb);
     p.ambbits = reinterpret_cast<unsigned *>(w + L.ambbits);
     p.p2w = reinterpret_cast<double *>(w + L.p2w);
+    p.p2lane = reinterpret_cast<double2 *>(w + L.p2lane);
 }
 
 // 2^(j/64), j = 0..63, from the host math library.
@@ -239,6 +250,28 @@ int launch_verify(Params &p, const Layout &L, void *ws, int dtype_index, cudaStr
         return SPEC_ECUDA;
     const int64_t blocks3 = std::max<int64_t>(1, std::min<int64_t>(sms, ceil_div(p.B, kWarps)));
     return launch_dependent(k_finalize<Tag, MODE>, blocks3, dyn3, st, p);
+}
+
+// The one-kernel linear path: clear the counters, then one resident wave.
+int g_fused_blocks[64][2];
+template <class Tag>
+int launch_fused(Params &p, const Layout &L, void *ws, int dtype_index, cudaStream_t st)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SPEC_ECUDA;
+    int per_sm, sms;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        per_sm = blocks_per_sm(g_fused_blocks[dev][dtype_index], k_fused<Tag>, kFusedSmem);
+        sms = sm_count(dev);
+    }
+    if (per_sm < 1 || sms < 1) return SPEC_ECUDA;
+    // counters and pass-1 partials to all ones (kPartEmpty), one contiguous range
+    const size_t clear = L.rowpart - L.counters + sizeof(float2) * static_cast<size_t>(p.nA);
+    if (cudaMemsetAsync(static_cast<char *>(ws) + L.counters, 0xFF, clear, st) != cudaSuccess)
+        return SPEC_ECUDA;
+    k_fused<Tag><<<static_cast<unsigned>(per_sm * sms), kThreads, kFusedSmem, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ECUDA;
 }
 
 // Largest number of co-resident greedy clusters, per device and dtype.
@@ -394,8 +427,8 @@ extern "C" int spec_verify_linear(const void *target_logits, const void *draft_l
     rc = setup_items(p, R, dtype, true);
     if (rc != SPEC_OK) return rc;
     fill_workspace(p, workspace, L);
-    return dtype == SPEC_BF16 ? launch_verify<Bf16, kLinear>(p, L, workspace, 1, stream)
-                              : launch_verify<F32, kLinear>(p, L, workspace, 0, stream);
+    return dtype == SPEC_BF16 ? launch_fused<Bf16>(p, L, workspace, 1, stream)
+                              : launch_fused<F32>(p, L, workspace, 0, stream);
 }
 
 extern "C" int spec_verify_greedy(const void *target_logits, spec_dtype_t dtype,

@@ -15,7 +15,7 @@ constexpr int kWarps = kThreads / 32;
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
 // Per-request status bits (mirror SPEC_STATUS_* in the public header).
-enum : int { kStToken = 1, kStTree = 2, kStLogit = 4 };
+enum : int { kStToken = 1, kStTree = 2, kStLogit = 4, kStTimeout = 8 };
 
 // Philox counter purposes.
 enum : uint32_t { kPurposeAccept = 0, kPurposeSample = 1 };
@@ -374,6 +374,11 @@ struct Params {
     int *p2amb;              // [B][S2] undecided entries per segment
     unsigned *ambbits;       // [B][W32] undecided entries, one bit each
     double *p2w;             // [B][2][S2] finalize scratch (vocabularies too large for shared memory)
+    double2 *p2lane;         // [B][S2][32] per-lane sums of pass 2 (decided part)
+    // one-kernel linear path (set to all ones per call, with rowpart)
+    unsigned *p2cnt;         // [B] pass-2 items completed per request
+    unsigned *p2claim;       // tasks claimed
+    unsigned *decided;       // [B] 1 once the request's decision is published
     double exp2tab[64];      // 2^(j/64), j = 0..63
 };
 

@@ -290,28 +290,30 @@ __device__ __forceinline__ float lane_max<F32>(const uint4 (&raw)[Pass1Shape<F32
     return m[0];
 }
 
-// Reduce one staged item and store its partial.  Stochastic: each lane
-// takes its own max m, then sums 2^(x c - fl(m c)): one FMA and one
+// Reduce one staged item (item id `item`, segment s of its row) and store
+// its partial at rowpart[item] (= rowpart[b][r][s]).  Stochastic: each
+// lane takes its own max m, then sums 2^(x c - fl(m c)): one FMA and one
 // special-function exponential per entry, four independent sums; the lane
-// sums are corrected for fl(m c) - m c and rescaled to the warp max.
+// sums are corrected by 2^(fl(m c) - m c) (the FMA residual gives the
+// difference exactly) and rescaled to the warp max.
 template <class Tag, int MODE>
-__device__ __forceinline__ void reduce_item1(const Params &p, const Item1 &it, const uint4 *slot)
+__device__ __forceinline__ void reduce_item1(const Params &p, unsigned item, int s, const uint4 *slot)
 {
     constexpr int kVec = Tag::kVec;
     constexpr int kV = Pass1Shape<Tag>::kVecL;
     const int lane = threadIdx.x & 31;
-    if (!it.active) return;
+    const int e_begin = s * Pass1Shape<Tag>::kItem;
     uint4 raw[kV];
-    if (it.e_begin + Pass1Shape<Tag>::kItem <= it.e_end) {
+    if (e_begin + Pass1Shape<Tag>::kItem <= p.V) {
 #pragma unroll
         for (int v = 0; v < kV; ++v) raw[v] = slot[v * 32 + lane];
     } else {  // the ragged end of a row
 #pragma unroll
         for (int v = 0; v < kV; ++v) {
-            const int e0 = it.e_begin + (v * 32 + lane) * kVec;
-            raw[v] = e0 < it.e_end ? mask_tail<Tag>(slot[v * 32 + lane], it.e_end - e0)
-                                   : make_uint4(Tag::kNegInfWord, Tag::kNegInfWord, Tag::kNegInfWord,
-                                                Tag::kNegInfWord);
+            const int e0 = e_begin + (v * 32 + lane) * kVec;
+            raw[v] = e0 < p.V ? mask_tail<Tag>(slot[v * 32 + lane], p.V - e0)
+                              : make_uint4(Tag::kNegInfWord, Tag::kNegInfWord, Tag::kNegInfWord,
+                                           Tag::kNegInfWord);
         }
     }
     float2 part;
@@ -323,7 +325,7 @@ __device__ __forceinline__ void reduce_item1(const Params &p, const Item1 &it, c
         for (int v = 0; v < kV; ++v) {
             float x[kVec];
             unpack<Tag>(raw[v], x);
-            const int e0 = it.e_begin + (v * 32 + lane) * kVec;
+            const int e0 = e_begin + (v * 32 + lane) * kVec;
 #pragma unroll
             for (int e = 0; e < kVec; ++e) {
                 nan |= (x[e] != x[e]);
@@ -358,16 +360,13 @@ __device__ __forceinline__ void reduce_item1(const Params &p, const Item1 &it, c
         const float M = warp_max_nan(m);
         float sr = 0.f;
         if (m != -INFINITY) {
-            // terms were taken against fl(m c); against m c they are
-            // larger by 2^(fl(m c) - m c) (an exact difference in fp64)
-            const float d = static_cast<float>(static_cast<double>(mc) -
-                                               static_cast<double>(m) * static_cast<double>(c));
-            sr = lsum * ex2_fma((m - M) * c) * fmaf(d, 0.693147180559945309f, 1.0f);
+            const float d = -fmaf(m, c, nmc);  // fl(m c) - m c, exactly
+            sr = lsum * ex2_approx((m - M) * c) * fmaf(d, 0.693147180559945309f, 1.0f);
         }
         sr = warp_sum(sr);
         part = make_float2(M, sr);
     }
-    if (lane == 0) __stcg(p.rowpart + (static_cast<int64_t>(it.b) * p.R + it.r) * p.S + it.s, part);
+    if (lane == 0) __stcg(p.rowpart + item, part);
 }
 
 // The pass-1 worker: warp w of W takes items w, w + W, w + 2W, ... (items
@@ -393,16 +392,19 @@ __device__ __forceinline__ void pass1_stream(const Params &p, uint4 *ring, unsig
     };
 #pragma unroll 1
     for (int q = 0; q < kRing1; ++q) refill(q);
+    // segment of the item in hand, advanced by W mod S per item
+    int s = static_cast<int>(w - fdiv(w, p.div_s) * static_cast<unsigned>(p.S));
+    const int ws = static_cast<int>(W - fdiv(W, p.div_s) * static_cast<unsigned>(p.S));
     int q = 0;
 #pragma unroll 1
     for (unsigned item = w; item < p.nA; item += W) {
         wait_copies<kRing1 - 1>();
-        if (__shfl_sync(kFull, act ? 1 : 0, q)) {
-            const Item1 it = item1<Tag, MODE>(p, item, false);
-            reduce_item1<Tag, MODE>(p, it, ring + q * kSlot);
-        }
+        if (MODE == kLinear || __shfl_sync(kFull, act ? 1 : 0, q))
+            reduce_item1<Tag, MODE>(p, item, s, ring + q * kSlot);
         refill(q);
         q = (q + 1 == kRing1) ? 0 : q + 1;
+        s += ws;
+        if (s >= p.S) s -= p.S;
     }
     wait_copies<0>();
 }
@@ -468,7 +470,6 @@ __device__ __forceinline__ void merge_row(const Params &p, int b, int r, RowStat
         if (lane == 0) {
             rs.m[r] = nan ? __int_as_float(0x7FC00000) : M;
             rs.s[r] = nan ? __longlong_as_double(0x7FF8000000000000ll) : S;
-            rs.idx[r] = 0;
         }
     }
 }
@@ -1048,9 +1049,9 @@ __device__ __forceinline__ int icdf_blocked(const double *W, int n, double u, do
 
 // Draw the token of request b by inverse CDF: segment weights (closed form
 // from the decided sums plus the exact weights of the marked entries), then
-// exact weights of the chosen segment's entries, read once (16 per lane):
-// lane sums pick the chunk, the owning lane walks it.  One warp; W, B: S2
-// doubles of scratch each.  The sums of a segment are read in one round.
+// the lane chunk of the chosen segment (the items' per-lane sums), then its
+// entries (exact weights, one per lane).  One warp; W, B: S2 doubles of
+// scratch each.  The sums of all segments are read in one round.
 template <class Tag>
 __device__ __forceinline__ void finalize(const Params &p, int b, const double *tab, double *W, double *B)
 {
@@ -1085,6 +1086,7 @@ __device__ __forceinline__ void finalize(const Params &p, int b, const double *t
         }
     }
     bool residual = info.mode == kModeResidual;
+    bool exact_lanes = false;
     double isp = 1.0, isq = 1.0;
     if (residual) {
         Sp = warp_sum(Sp);
@@ -1094,6 +1096,7 @@ __device__ __forceinline__ void finalize(const Params &p, int b, const double *t
         const double rho = Sp / Sq;
         __syncwarp();
         if (!(rho >= info.rho_lo && rho <= info.rho_hi)) {
+            exact_lanes = true;
             // the pass-1 estimate missed: every weight exactly, a segment at a time
             for (int s = 0; s < S2; ++s) {
                 const double w =
@@ -1119,6 +1122,7 @@ __device__ __forceinline__ void finalize(const Params &p, int b, const double *t
         for (int s = lane; s < S2; s += 32) z += W[s];
         if (!(warp_sum(z) > 0.0)) {  // residual mass vanished in rounding: draw from target row n
             residual = false;
+            exact_lanes = true;  // the items' lane sums are residual sums
             __syncwarp();
             for (int s = lane; s < S2; s += 32) W[s] = ldcg_d4(part + s).x;
         }
@@ -1129,10 +1133,28 @@ __device__ __forceinline__ void finalize(const Params &p, int b, const double *t
     if (sstar < 0) sstar = 0;
     const double tseg = info.u * Z - before;
 
-    // the chosen segment: exact weights, 16 entries per lane
-    double wl[kLane2];
-    const double lane_w =
-        lane_exact_weights<Tag>(p, info, residual, sstar * kSeg2 + lane * kLane2, isp, isq, tab, wl);
+    // lane chunks of the chosen segment: the items' per-lane sums of the
+    // decided entries plus the exact weights of the lane's marked entries
+    // (every entry exactly when the pass-1 estimate missed or the residual
+    // vanished)
+    const int clo = sstar * kSeg2 + lane * kLane2;
+    double lane_w;
+    if (exact_lanes) {
+        lane_w = lane_exact_sum<Tag>(p, info, residual, clo, isp, isq, tab);
+    } else {
+        const double2 pl = __ldcg(p.p2lane + (static_cast<int64_t>(b) * S2 + sstar) * 32 + lane);
+        if (residual) {
+            const double w = pl.x * isp - pl.y * isq;
+            lane_w = w > 0.0 ? w : 0.0;
+            if (__ldcg(namb + sstar) > 0) {
+                // this lane's 16 entries are one half of bitmap word clo / 32
+                const unsigned keep = (clo & 31) ? 0xFFFF0000u : 0x0000FFFFu;
+                lane_w += marked_sum<Tag, 1>(p, info, bits, clo >> 5, keep, isp, isq, tab);
+            }
+        } else {
+            lane_w = pl.x;
+        }
+    }
     const double incl = warp_incl_scan(lane_w);
     double excl = __shfl_up_sync(kFull, incl, 1);
     if (lane == 0) excl = 0.0;
@@ -1145,22 +1167,22 @@ __device__ __forceinline__ void finalize(const Params &p, int b, const double *t
         cl = pos ? 31 - __clz(pos) : 0;
     }
     const double tchunk = tseg - __shfl_sync(kFull, excl, cl);
-    int e_hit = -1, e_last = -1;
-    if (lane == cl) {
-        double run = 0.0;
-#pragma unroll
-        for (int e = 0; e < kLane2; ++e) {
-            run += wl[e];
-            if (wl[e] > 0.0) {
-                e_last = e;
-                if (e_hit < 0 && run > tchunk) e_hit = e;
-            }
-        }
+
+    // entries of chunk cl, one per lane
+    const int cbase = sstar * kSeg2 + cl * kLane2;
+    const int idx = cbase + lane;
+    const bool valid = lane < kLane2 && idx < p.V;
+    const double w1 = valid ? exact_weight<Tag>(p, info, residual, idx, isp, isq, tab) : 0.0;
+    const double pincl = warp_incl_scan(w1);
+    const unsigned ehit = __ballot_sync(kFull, w1 > 0.0 && pincl > tchunk);
+    int token;
+    if (ehit) {
+        token = cbase + __ffs(ehit) - 1;
+    } else {
+        const unsigned pos = __ballot_sync(kFull, w1 > 0.0);
+        token = pos ? cbase + 31 - __clz(pos) : cbase;
     }
-    e_hit = __shfl_sync(kFull, e_hit, cl);
-    e_last = __shfl_sync(kFull, e_last, cl);
-    const int e_tok = e_hit >= 0 ? e_hit : (e_last >= 0 ? e_last : 0);
-    if (lane == 0) p.out[info.out_index] = sstar * kSeg2 + cl * kLane2 + e_tok;
+    if (lane == 0) p.out[info.out_index] = token;
 }
 
 // One pass-2 item: reduce, then publish the sums, the per-lane partials
@@ -1172,6 +1194,7 @@ __device__ __forceinline__ void p2_item(const Params &p, int b, int s2, const It
     const int lane = threadIdx.x & 31;
     const P2Acc a = reduce_item<Tag, kResidual>(p, it, s2, buf, tab);
     const int64_t at = static_cast<int64_t>(b) * p.S2 + s2;
+    __stcg(p.p2lane + at * 32 + lane, make_double2(a.A, a.B));
     int namb = 0;
     if (kResidual) {
         // two lanes' 16-entry masks form one bitmap word
