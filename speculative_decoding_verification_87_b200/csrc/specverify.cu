@@ -75,8 +75,8 @@ Layout layout(int B, int R, int V)
     const int64_t s2 = ceil_div(V, kSeg2);
     const int64_t w32 = s2 * (kSeg2 / 32);  // whole segments (16-byte aligned rows of the bitmap)
     size_t off = 0;
-    L.counters = off;  // p2cnt[B], decided[B], p2claim; rowpart follows directly
-    off = align_up(off + sizeof(unsigned) * (2 * static_cast<size_t>(B) + 1));
+    L.counters = off;  // p2cnt[B], decided[B], p2claim, a_claim; rowpart follows directly
+    off = align_up(off + sizeof(unsigned) * (2 * static_cast<size_t>(B) + 2));
     L.rowpart = off;
     off = align_up(off + sizeof(float2) * static_cast<size_t>(B) * R * smax);
     L.req = off;
@@ -124,6 +124,7 @@ void fill_workspace(Params &p, void *ws, const Layout &L)
     p.p2cnt = cnt;
     p.decided = cnt + p.B;
     p.p2claim = p.decided + p.B;
+    p.a_claim = p.p2claim + 1;
     p.rowpart = reinterpret_cast<float2 *>(w + L.rowpart);
     p.req = reinterpret_cast<ReqInfo *>(w + L.req);
     p.p2part = reinterpret_cast<double4 *>(w + L.p2part);
@@ -266,6 +267,9 @@ int launch_fused(Params &p, const Layout &L, void *ws, int dtype_index, cudaStre
         sms = sm_count(dev);
     }
     if (per_sm < 1 || sms < 1) return SPEC_ECUDA;
+    // whole static rounds for about the first 88% of the pass-1 items
+    const unsigned W = static_cast<unsigned>(per_sm * sms * kStreamers);
+    p.nAs = static_cast<unsigned>((static_cast<uint64_t>(p.nA) * 88 / 100) / W * W);
     // counters and pass-1 partials to all ones (kPartEmpty), one contiguous range
     const size_t clear = L.rowpart - L.counters + sizeof(float2) * static_cast<size_t>(p.nA);
     if (cudaMemsetAsync(static_cast<char *>(ws) + L.counters, 0xFF, clear, st) != cudaSuccess)

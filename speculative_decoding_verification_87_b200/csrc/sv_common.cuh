@@ -378,6 +378,8 @@ struct Params {
     // one-kernel linear path (set to all ones per call, with rowpart)
     unsigned *p2cnt;         // [B] pass-2 items completed per request
     unsigned *p2claim;       // tasks claimed
+    unsigned *a_claim;       // pass-1 chunks claimed past nAs
+    unsigned nAs;            // pass-1 items taken in static round robin
     unsigned *decided;       // [B] 1 once the request's decision is published
     double exp2tab[64];      // 2^(j/64), j = 0..63
 };

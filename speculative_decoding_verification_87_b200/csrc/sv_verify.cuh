@@ -917,10 +917,11 @@ __device__ __forceinline__ double marked_sum(const Params &p, const ReqInfo &inf
                                              int w0, unsigned keep, double isp, double isq, const double *tab)
 {
     unsigned m[kWords];
-    if (kWords == 16) {
+    if constexpr (kWords > 1) {
+        static_assert(kWords % 4 == 0, "whole 16-byte words");
         const uint4 *q = reinterpret_cast<const uint4 *>(bits + w0);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < kWords / 4; ++i) {
             const uint4 u = __ldcg(q + i);
             m[4 * i] = u.x;
             m[4 * i + 1] = u.y;
@@ -1114,7 +1115,7 @@ __device__ __forceinline__ void finalize(const Params &p, int b, const double *t
                 marked &= marked - 1;
                 for (int s = j * 32 + lane; s < S2; s += 32 * 32)
                     if (__ldcg(namb + s) > 0)
-                        W[s] += marked_sum<Tag, 16>(p, info, bits, s * (kSeg2 / 32), 0u, isp, isq, tab);
+                        W[s] += marked_sum<Tag, kSeg2 / 32>(p, info, bits, s * (kSeg2 / 32), 0u, isp, isq, tab);
             }
         }
         __syncwarp();
@@ -1147,8 +1148,9 @@ __device__ __forceinline__ void finalize(const Params &p, int b, const double *t
             const double w = pl.x * isp - pl.y * isq;
             lane_w = w > 0.0 ? w : 0.0;
             if (__ldcg(namb + sstar) > 0) {
-                // this lane's 16 entries are one half of bitmap word clo / 32
-                const unsigned keep = (clo & 31) ? 0xFFFF0000u : 0x0000FFFFu;
+                // this lane's entries: the bits of [clo, clo + kLane2) of word clo / 32
+                static_assert(kLane2 == 16 || kLane2 == 32, "a lane's entries lie in one bitmap word");
+                const unsigned keep = kLane2 == 32 ? 0xFFFFFFFFu : ((clo & 31) ? 0xFFFF0000u : 0x0000FFFFu);
                 lane_w += marked_sum<Tag, 1>(p, info, bits, clo >> 5, keep, isp, isq, tab);
             }
         } else {
@@ -1197,12 +1199,15 @@ __device__ __forceinline__ void p2_item(const Params &p, int b, int s2, const It
     __stcg(p.p2lane + at * 32 + lane, make_double2(a.A, a.B));
     int namb = 0;
     if (kResidual) {
-        // two lanes' 16-entry masks form one bitmap word
-        static_assert(kLane2 == 16, "bitmap words hold two lanes' entries");
-        const unsigned other = __shfl_down_sync(kFull, a.amb, 1);
         const int word = (s2 * kSeg2 + lane * kLane2) >> 5;
-        if (!(lane & 1) && word < p.W32)
-            __stcg(p.ambbits + static_cast<int64_t>(b) * p.W32 + word, a.amb | (other << 16));
+        if constexpr (kLane2 == 32) {
+            __stcg(p.ambbits + static_cast<int64_t>(b) * p.W32 + word, a.amb);
+        } else {
+            // two lanes' 16-entry masks form one bitmap word
+            static_assert(kLane2 == 16, "one or two lanes per bitmap word");
+            const unsigned other = __shfl_down_sync(kFull, a.amb, 1);
+            if (!(lane & 1)) __stcg(p.ambbits + static_cast<int64_t>(b) * p.W32 + word, a.amb | (other << 16));
+        }
         namb = __popc(a.amb);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) namb += __shfl_xor_sync(kFull, namb, o);
