@@ -31,7 +31,42 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "verify rows/s and achieved HBM GB/s (B=64, k=8, V=128256 bf16, 1 B200)"
+# the kernels one call launches, per workload
+KERNEL_OF = {
+    "batched": "k_fused (one launch per call, after a 0.55 MB memset)",
+    "single": "k_fused (one launch per call, after a memset)",
+    "greedy": "k_greedy_cluster (one launch per call)",
+    "tree": "k_pass1 + k_decide (programmatic dependents)",
+    "tree-stochastic": "k_pass1 + k_decide + k_pass2 + k_finalize (programmatic dependents)",
+}
 L2_BYTES = 126 * 2 ** 20
+
+
+def csrc_digest():
+    """sha256 over the CUDA sources (sorted by name): identifies the kernels."""
+    import hashlib
+    d = os.path.join(ROOT, "speculative_decoding_verification_87_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh")):
+            h.update(name.encode())
+            with open(os.path.join(d, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary (profiles/traffic.json), or None when the kernels have changed
+    since those counters were taken."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            entry = json.load(f).get(workload)
+    except Exception:
+        return None, None
+    if not entry or entry.get("csrc_sha256") != csrc_digest():
+        return None, None
+    return entry["dram_read_bytes"] + entry["dram_write_bytes"], entry.get("summary")
 
 
 def _peaks():
@@ -194,6 +229,16 @@ def barrier(world):
         dist.barrier()
 
 
+def shard_seeds(rank, nsets=2):
+    """Seeds of a rank's resident input sets: ranks verify disjoint requests."""
+    return [1000 * rank + s for s in range(nsets)]
+
+
+def whole_job_rate(rows_per_step, steps, world, ms_max):
+    """Rows per second of the whole job: every rank's rows over the slowest rank's time."""
+    return rows_per_step * steps * world / (ms_max / 1e3)
+
+
 # -------------------------------------------------------------- our arm
 class Runner:
     """Binds one workload's device buffers to the C-ABI call of its mode."""
@@ -222,8 +267,8 @@ class Runner:
         else:
             self.tokens = dev(w.tokens.astype(np.int32))
             self.out = torch.empty((w.batch, w.k + 1), dtype=torch.int32, device=device)
-            # greedy: one cluster kernel; linear: pass 1, decide, pass 2, finalize
-            self.kernels_per_call = 1 if name == "greedy" else 4
+            # greedy: the cluster kernel; linear stochastic: k_fused
+            self.kernels_per_call = 1
         self.acc = torch.empty((w.batch,), dtype=torch.int32, device=device)
 
     def call(self, offset, target=None, draft=None, tokens=None):
@@ -252,7 +297,7 @@ def run_ours(args, rank, world, local):
     binding.load_library()
     device = torch.device("cuda", local)
     name = args.config
-    sets = [make_workload(name, seed=1000 * rank + s) for s in range(2)]
+    sets = [make_workload(name, seed=s) for s in shard_seeds(rank)]
     rows, alg_bytes, cfg = workload_facts(name, sets[0])
     runners = [Runner(name, w, device) for w in sets]
     stream = torch.cuda.current_stream(device)
@@ -277,10 +322,11 @@ def run_ours(args, rank, world, local):
         barrier(world)
     ms = start.elapsed_time(stop)
     ms_max = max_over_ranks(ms, world, device)
-    value = rows * args.steps * world / (ms_max / 1e3)
+    value = whole_job_rate(rows, args.steps, world, ms_max)
     step_s = ms_max / 1e3 / args.steps
     peak, peak_src = _peaks()
     achieved = alg_bytes / step_s / 1e9
+    traffic, traffic_src = measured_traffic(cfg["workload"])
 
     # end to end through the same API from pinned host buffers: each step
     # copies its inputs host->device, verifies, and reads the outputs back
@@ -305,10 +351,13 @@ def run_ours(args, rank, world, local):
                               f"{alg_bytes / 1e6:.1f} MB alternate",
                            requests_per_rank=sets[0].batch),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None,
+                         "frac": achieved / peak, "traffic": traffic,
+                         "traffic_source": traffic_src,
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
                          if peak_src == "measured" else "fallback",
-                         "kernel": "whole verification call (all kernels of a step)",
+                         "kernel": KERNEL_OF.get(name, "verification call"),
+                         "timed": "CUDA events around each call on its stream (all of the call's "
+                                  "kernels, which run back to back)",
                          "algorithmic_bytes_per_launch": alg_bytes},
             "e2e": e2e,
             "gpu_launches": runners[0].kernels_per_call * args.steps,
