@@ -172,3 +172,53 @@ def test_tiny_config_1e6_trials(sv, orc):
             counts = np.bincount(out[sel, j], minlength=base.vocab)
             pv, bad = chisquare_pvalue(counts, p[b, j])
             assert bad == 0 and pv > 1e-3, (b, j, pv)
+
+
+def test_near_identical_rows_mark_many_entries(sv, orc):
+    """Draft rows within ~1% of the target rows: residual draws whose p - q
+    sign is undecided from fp32 for many entries (resolved exactly)."""
+    w = wl.peaked_linear(seed=31, batch=32, k=32, vocab=20000, temperature=1.0,
+                         sigma=(0.02, 0.02), dtype="f32")
+    residual = 0
+    for off in range(3):
+        g = run_linear_gpu(sv, w, seed=5, offset=off)
+        o = orc.verify_linear(w.target, w.draft, w.tokens, w.vocab, w.temperature, 5, off)
+        assert g["status"] == 0
+        compare_linear(g, o, w.k)
+        residual += int(np.sum(g["acc"] < w.k))
+    assert residual > 0
+
+
+def test_masked_vocabulary_is_never_drawn(sv, orc):
+    """-inf logits (a masked tail and scattered holes) in both rows."""
+    w = wl.peaked_linear(seed=41, batch=24, k=4, vocab=20000, temperature=0.9,
+                         sigma=(0.5, 2.0), dtype="bf16")
+    V = w.vocab
+    rng = np.random.default_rng(7)
+    holes = rng.choice(15000, size=500, replace=False)
+    t, d = w.target.copy(), w.draft.copy()
+    for a in (t, d):
+        a[..., 15000:V] = np.uint16(0xFF80)
+        a[..., holes] = np.uint16(0xFF80)
+    w.target, w.draft = t, d
+    w.tokens = wl.gumbel_max(rng, wl.as_f32(d, V), w.temperature).astype(np.int32)
+    masked = np.zeros(V, bool)
+    masked[15000:] = True
+    masked[holes] = True
+    for off in range(4):
+        g = run_linear_gpu(sv, w, seed=9, offset=off)
+        o = orc.verify_linear(w.target, w.draft, w.tokens, w.vocab, w.temperature, 9, off)
+        assert g["status"] == 0
+        compare_linear(g, o, w.k)
+        out = g["out"]
+        assert not np.any(masked[out[out >= 0]])
+
+
+def test_more_requests_than_task_warps(sv, orc):
+    """B = 700: the decide tasks outnumber the warps that take tasks first."""
+    w = wl.peaked_linear(seed=51, batch=700, k=3, vocab=2000, temperature=1.0,
+                         sigma=(0.5, 2.0), dtype="bf16")
+    g = run_linear_gpu(sv, w, seed=11, offset=0)
+    o = orc.verify_linear(w.target, w.draft, w.tokens, w.vocab, w.temperature, 11, 0)
+    assert g["status"] == 0
+    compare_linear(g, o, w.k)
