@@ -323,6 +323,11 @@ def run_ours(args, rank, world, local):
     ms = start.elapsed_time(stop)
     ms_max = max_over_ranks(ms, world, device)
     value = whole_job_rate(rows, args.steps, world, ms_max)
+    # tokens a call emits (accepted drafts + the drawn token), from each
+    # input set's last call
+    acc = np.concatenate([r.acc.cpu().numpy() for r in runners])
+    emitted_per_step = float(np.mean(acc + 1)) * acc.size / len(runners)
+    tokens_per_s = whole_job_rate(emitted_per_step, args.steps, world, ms_max)
     step_s = ms_max / 1e3 / args.steps
     peak, peak_src = _peaks()
     achieved = alg_bytes / step_s / 1e9
@@ -362,7 +367,8 @@ def run_ours(args, rank, world, local):
             "e2e": e2e,
             "gpu_launches": runners[0].kernels_per_call * args.steps,
             "clocks": clk.summary(),
-            "tokens_per_s": None,
+            "tokens_per_s": tokens_per_s,
+            "mean_accepted": float(np.mean(acc)),
         }
         if args.cpu_baseline and world == 1:
             line["cpu_baseline"] = oracle_baseline(name, sets[0], rows)

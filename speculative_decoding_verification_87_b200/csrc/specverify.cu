@@ -1,11 +1,13 @@
 // specverify.cu -- C ABI of libspecverify.so (sm_100a) and its launches.
 //
-// spec_verify_linear / spec_verify_tree: the pass-1 kernel, the decide
-// kernel and, where a token is drawn, the pass-2 and finalize kernels
-// (sv_verify.cuh), each a programmatic dependent of the one before, on the
-// caller's stream; no host synchronisation and no workspace clearing.
+// spec_verify_linear: one memset of the call's counters and pass-1
+// partials, then the persistent kernel k_fused (sv_fused.cuh).
+// spec_verify_tree: the pass-1 kernel, the decide kernel and, where a token
+// is drawn, the pass-2 and finalize kernels (sv_verify.cuh), each a
+// programmatic dependent of the one before.
 // spec_verify_greedy: one launch of the cluster kernel (sv_greedy.cuh); no
 // workspace.
+// Everything is enqueued on the caller's stream; no host synchronisation.
 #include <algorithm>
 #include <climits>
 #include <cmath>

@@ -222,10 +222,6 @@ __device__ __forceinline__ void argmax_take(float &bv, int &bi, float ov, int oi
     }
 }
 
-__device__ __forceinline__ unsigned ld_volatile(const unsigned *p)
-{
-    return *reinterpret_cast<const volatile unsigned *>(p);
-}
 
 // ---------------------------------------------------------------- reductions
 __device__ __forceinline__ float warp_max_nan(float v)
@@ -257,69 +253,6 @@ __device__ __forceinline__ int warp_max(int v)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(kFull, v, o));
     return v;
-}
-
-// Block-wide reductions over kThreads threads; every thread gets the result.
-// `red` is shared scratch of at least kWarps elements of the value type.
-__device__ __forceinline__ float block_max_nan(float v, float *red)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    v = warp_max_nan(v);
-    __syncthreads();
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    float r = red[0];
-#pragma unroll
-    for (int w = 1; w < kWarps; ++w) r = max_nan(r, red[w]);
-    return r;
-}
-__device__ __forceinline__ float block_sum(float v, float *red)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    v = warp_sum(v);
-    __syncthreads();
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    float r = red[0];
-#pragma unroll
-    for (int w = 1; w < kWarps; ++w) r += red[w];
-    return r;
-}
-__device__ __forceinline__ double block_sum(double v, double *red)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    v = warp_sum(v);
-    __syncthreads();
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    double r = red[0];
-#pragma unroll
-    for (int w = 1; w < kWarps; ++w) r += red[w];
-    return r;
-}
-__device__ __forceinline__ int block_min(int v, int *red)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    v = warp_min(v);
-    __syncthreads();
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    int r = red[0];
-#pragma unroll
-    for (int w = 1; w < kWarps; ++w) r = min(r, red[w]);
-    return r;
-}
-__device__ __forceinline__ int block_max(int v, int *red)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    v = warp_max(v);
-    __syncthreads();
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    int r = red[0];
-#pragma unroll
-    for (int w = 1; w < kWarps; ++w) r = max(r, red[w]);
-    return r;
 }
 
 // ------------------------------------------------------- per-call parameters

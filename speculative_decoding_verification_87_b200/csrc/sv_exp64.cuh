@@ -46,18 +46,5 @@ __device__ __forceinline__ double exp2_fp64(double z, const double *tab)
     return z > -1020.0 ? y : 0.0;
 }
 
-// Exact widening of a bf16 bit pattern (low 16 bits of h) to fp64 with
-// integer operations only; subnormal values become signed zero (no fp64
-// quantity here can tell them apart), infinities and NaN keep their class.
-__device__ __forceinline__ double bf16_to_f64(uint32_t h)
-{
-    const uint32_t sign = (h & 0x8000u) << 16;
-    const uint32_t e = (h >> 7) & 0xFFu;
-    const uint32_t m = (h & 0x7Fu) << 13;
-    const uint32_t hi = e == 0xFFu ? (sign | 0x7FF00000u | m)
-                      : e == 0u    ? sign
-                                   : (sign | ((e + 896u) << 20) | m);
-    return __hiloint2double(static_cast<int>(hi), 0);
-}
 
 }  // namespace sv

@@ -1,34 +1,34 @@
-// sv_verify.cuh -- the verification path as two kernels (linear
-// stochastic, tree stochastic, tree greedy).
+// sv_verify.cuh -- the steps of stochastic and tree verification, and the
+// four-kernel path of the tree modes (the linear mode runs the same steps
+// in one kernel, sv_fused.cuh).
 //
-//  * k_pass1 (items of `seg` entries of one logit row, request-major
-//    order, claimed by fetch-and-add): one streaming read of every row,
-//    moved by asynchronous copies into a per-warp shared-memory ring kRing
-//    batches ahead of use.  Stochastic modes reduce an item to (max,
-//    sum exp((l - max)/T)), three quarters of the exponentials on the
-//    special-function unit and one quarter on the FMA pipe; greedy trees
-//    reduce to (max, lowest argmax).  "Accelerating Sonar through
-//    speculation", section "Target-Draft": acceptance compares the full
-//    draft and target distributions, hence whole-vocabulary normalisers.
-//    The warp that completes the last item of a row merges the row; the
-//    warp that merges the last row of a request runs the request's decide
-//    step ("Speculative decoding explained", section "Draft and
-//    verification loop"; section "EAGLE" of the Sonar post for trees).
-//  * k_pass2 (items of kSeg2 entries of the row, or row pair, that the final
-//    draw needs): fp64 weights.  For the residual norm(max(0, p_n - q_n))
+//  * Pass 1 (k_pass1): one streaming read of every row that a mode needs,
+//    in items of 2048 bf16 (1024 fp32) entries of one row taken by warps in
+//    static round robin and copied by asynchronous copies into a per-warp
+//    shared-memory ring ahead of use.  Stochastic modes reduce an item to
+//    (max, sum exp((l - max)/T)) with one special-function exponential per
+//    entry; greedy trees reduce to (max, lowest argmax).  "Accelerating
+//    Sonar through speculation", section "Target-Draft": acceptance
+//    compares the full draft and target distributions, hence
+//    whole-vocabulary normalisers.
+//  * Decide (k_decide): one block per request merges its rows' partials
+//    and runs the decide step ("Speculative decoding explained", section
+//    "Draft and verification loop"; section "EAGLE" of the Sonar post for
+//    trees).
+//  * Pass 2 (k_pass2): items of kSeg2 entries of the row, or row pair, that
+//    the final draw needs, in fp64.  For the residual norm(max(0, p_n - q_n))
 //    one pass yields both normalisers and the segment sums: an entry whose
-//    sign of p - q is already decided by the fp32 ratio bounds goes into a
+//    sign of p - q is already certain from its fp32 logits goes into a
 //    linear sum, the few undecided ones are marked in a bitmap and resolved
 //    exactly once the fp64 normalisers are known.  Per-lane partial sums
-//    are kept, so the warp that completes the last pass-2 item of a request
-//    draws the token by inverse CDF (segment prefix, lane-chunk prefix,
-//    entry) without recomputing the chosen segment.
+//    are kept for the draw.
+//  * Finalize (k_finalize): one warp per request draws the token by inverse
+//    CDF (segment, lane chunk, entry).
 //
-// k_pass2 is a programmatic dependent of k_pass1: its blocks are scheduled
-// as pass-1 blocks retire and start work once pass 1 has completed and its
-// writes are visible.  No warp ever waits on another warp's progress; the
-// only waits are hardware waits (own asynchronous copies, the grid
-// dependency).
+// Each kernel is a programmatic dependent of the one before: its blocks are
+// scheduled as the previous grid's retire and start work once that grid
+// has completed and its writes are visible.  The only waits are hardware
+// waits (own asynchronous copies, the grid dependency).
 #pragma once
 
 #include "sv_common.cuh"
@@ -164,7 +164,6 @@ struct Pass1Shape {
 constexpr int kRing1 = 3;  // ring slots per warp: one reduced, two in flight
 constexpr size_t kRingBytes = sizeof(uint4) * kRing1 * 32 * 8 * kWarps;
 constexpr unsigned kNoItem = 0xFFFFFFFFu;
-constexpr unsigned kIdleItem = 0x80000000u;  // slot meta flag: the row is not read
 
 struct Item1 {
     const char *row;
@@ -858,55 +857,6 @@ __device__ __forceinline__ double lane_exact_sum(const Params &p, const ReqInfo 
     return w;
 }
 
-// Exact weights of this lane's kLane2 entries [lo, lo + kLane2) into w[],
-// read as whole vectors; returns their sum in index order.
-template <class Tag>
-__device__ __forceinline__ double lane_exact_weights(const Params &p, const ReqInfo &info, bool residual, int lo,
-                                                     double isp, double isq, const double *tab,
-                                                     double (&w)[kLane2])
-{
-    constexpr int kVec = Tag::kVec;
-    constexpr int kEsz = sizeof(typename Tag::elem);
-    constexpr int kNV = kLane2 / kVec;
-    const char *trow = static_cast<const char *>(p.tl) + info.t_off * kEsz;
-    const char *drow = static_cast<const char *>(p.dl) + info.d_off * kEsz;
-    const double nmt = neg_mc(p, info.mt), nmd = neg_mc(p, info.md);
-    uint4 tv[kNV], dv[kNV];
-#pragma unroll
-    for (int v = 0; v < kNV; ++v) {
-        const int e0 = lo + v * kVec;
-        const bool in = e0 < p.V;
-        tv[v] = in ? __ldcg(reinterpret_cast<const uint4 *>(trow + static_cast<int64_t>(e0) * kEsz))
-                   : make_uint4(0, 0, 0, 0);
-        dv[v] = (in && residual) ? __ldcg(reinterpret_cast<const uint4 *>(drow + static_cast<int64_t>(e0) * kEsz))
-                                 : make_uint4(0, 0, 0, 0);
-    }
-    double sum = 0.0;
-#pragma unroll
-    for (int v = 0; v < kNV; ++v) {
-        const int e0 = lo + v * kVec;
-        if (e0 + kVec > p.V) {
-            tv[v] = mask_tail<Tag>(tv[v], p.V - e0);
-            dv[v] = mask_tail<Tag>(dv[v], p.V - e0);
-        }
-        float xt[kVec], xd[kVec];
-        unpack<Tag>(tv[v], xt);
-        unpack<Tag>(dv[v], xd);
-#pragma unroll
-        for (int e = 0; e < kVec; ++e) {
-            const double et = exp2_fp64(entry_z(p, xt[e], nmt), tab);
-            double we = et;
-            if (residual) {
-                const double ef = exp2_fp64(entry_z(p, xd[e], nmd), tab);
-                const double pp = et * isp, qq = ef * isq;
-                we = pp > qq ? pp - qq : 0.0;
-            }
-            w[v * kVec + e] = we;
-            sum += we;
-        }
-    }
-    return sum;
-}
 
 // Exact weights, summed in index order, of the marked entries among the
 // n32 bitmap words starting at word w0 (n32 = 16: a whole segment, read as
