@@ -11,7 +11,7 @@
 // rank-0 block merges the CL partials through distributed shared memory,
 // scans for the first mismatch and writes the outputs.  Partials are double
 // buffered, so one barrier per request suffices.  Clusters stride over the
-// batch.
+// batch; a block's reads run one step ahead of its reductions and barriers.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -31,6 +31,7 @@ __global__ void __launch_bounds__(kThreads) k_greedy_cluster(const Params p, int
     constexpr int kVec = Tag::kVec;
     constexpr int kEsz = sizeof(typename Tag::elem);
     constexpr int U = 4;
+    constexpr int kChunk = kThreads * kVec * U;  // entries of a slice read per step
 
     __shared__ float2 part[2][kMaxRowsGreedy];
     __shared__ float redf[kWarps];
@@ -42,41 +43,62 @@ __global__ void __launch_bounds__(kThreads) k_greedy_cluster(const Params p, int
     const int cid = blockIdx.x / CL, ncl = gridDim.x / CL;
     const int k = p.k, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int s_begin = min(p.V, rank * slice), s_end = min(p.V, s_begin + slice);
+    // steps per row (an empty slice still takes one, so every row is reduced)
+    const int iters = max(1, (s_end - s_begin + kChunk - 1) / kChunk);
 
-    int it = 0;
-    for (int b = cid; b < p.B; b += ncl, ++it) {
-        const int buf = it & 1;
-        for (int j = 0; j <= k; ++j) {
-            const char *row = static_cast<const char *>(p.tl) +
-                              (static_cast<int64_t>(b) * (k + 1) + j) * p.stride * kEsz;
-            float best = -INFINITY;
-            int idx = INT_MAX;
-            bool nan = false;
-            for (int base = s_begin; base < s_end; base += kThreads * kVec * U) {
-                uint4 raw[U];
+    // The block's steps form one sequence over (request, row, step); the
+    // loads of the next step are issued before the current one is reduced,
+    // so they overlap the reduction and the block and cluster barriers.
+    auto load = [&](int b, int j, int it, uint4 (&raw)[U]) {
+        const char *row = static_cast<const char *>(p.tl) +
+                          (static_cast<int64_t>(b) * (k + 1) + j) * p.stride * kEsz;
+        const int base = s_begin + it * kChunk;
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const int e0 = base + (tid + u * kThreads) * kVec;
-                    raw[u] = e0 < s_end ? ldg_vec(row + static_cast<int64_t>(e0) * kEsz)
-                                        : make_uint4(Tag::kNegInfWord, Tag::kNegInfWord,
-                                                     Tag::kNegInfWord, Tag::kNegInfWord);
-                }
+        for (int u = 0; u < U; ++u) {
+            const int e0 = base + (tid + u * kThreads) * kVec;
+            raw[u] = e0 < s_end ? ldg_vec(row + static_cast<int64_t>(e0) * kEsz)
+                                : make_uint4(Tag::kNegInfWord, Tag::kNegInfWord, Tag::kNegInfWord,
+                                             Tag::kNegInfWord);
+        }
+    };
+    int b = cid, j = 0, it = 0;
+    uint4 cur[U], nxt[U];
+    if (b < p.B) load(b, j, it, cur);
+    float best = -INFINITY;
+    int idx = INT_MAX;
+    bool nan = false;
+    int rq = 0;  // requests done by this cluster (parity selects the partials buffer)
+#pragma unroll 1
+    while (b < p.B) {
+        // the step after this one
+        int nb = b, nj = j, nit = it + 1;
+        if (nit == iters) {
+            nit = 0;
+            if (++nj > k) {
+                nj = 0;
+                nb += ncl;
+            }
+        }
+        if (nb < p.B) load(nb, nj, nit, nxt);
+        const int base = s_begin + it * kChunk;
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const int e0 = base + (tid + u * kThreads) * kVec;
-                    if (e0 < s_end && e0 + kVec > s_end) raw[u] = mask_tail<Tag>(raw[u], s_end - e0);
-                    float x[kVec];
-                    unpack<Tag>(raw[u], x);
+        for (int u = 0; u < U; ++u) {
+            const int e0 = base + (tid + u * kThreads) * kVec;
+            uint4 raw = cur[u];
+            if (e0 < s_end && e0 + kVec > s_end) raw = mask_tail<Tag>(raw, s_end - e0);
+            float x[kVec];
+            unpack<Tag>(raw, x);
 #pragma unroll
-                    for (int e = 0; e < kVec; ++e) {
-                        nan |= (x[e] != x[e]);
-                        if (x[e] > best) {
-                            best = x[e];
-                            idx = e0 + e;
-                        }
-                    }
+            for (int e = 0; e < kVec; ++e) {
+                nan |= (x[e] != x[e]);
+                if (x[e] > best) {
+                    best = x[e];
+                    idx = e0 + e;
                 }
             }
+        }
+        if (it == iters - 1) {  // row j of request b is reduced: merge the block
+            const int buf = rq & 1;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 const float ov = __shfl_xor_sync(kFull, best, o);
@@ -93,52 +115,61 @@ __global__ void __launch_bounds__(kThreads) k_greedy_cluster(const Params p, int
                 float bv = redf[0];
                 int bi = redi[0];
                 for (int w = 1; w < kWarps; ++w) argmax_take(bv, bi, redf[w], redi[w]);
-                part[buf][j] = make_float2(any_nan ? __int_as_float(0x7FC00000) : bv,
-                                           __int_as_float(bi));
+                part[buf][j] = make_float2(any_nan ? __int_as_float(0x7FC00000) : bv, __int_as_float(bi));
             }
             __syncthreads();
+            best = -INFINITY;
+            idx = INT_MAX;
+            nan = false;
+            if (j == k) {  // the request is reduced in every block of the cluster
+                cluster.sync();
+                if (rank == 0) {
+                    if (tid == 0) nan_sh = 0;
+                    __syncthreads();
+                    for (int jj = tid; jj <= k; jj += kThreads) {
+                        float bv = -INFINITY;
+                        int bi = INT_MAX;
+                        bool nn = false;
+                        for (int r = 0; r < CL; ++r) {  // slices in index order
+                            const float2 *rp = cluster.map_shared_rank(&part[buf][0], r);
+                            const float2 v = rp[jj];
+                            if (v.x != v.x) nn = true;
+                            else argmax_take(bv, bi, v.x, __float_as_int(v.y));
+                        }
+                        if (nn) atomicOr(&nan_sh, 1);
+                        g_sh[jj] = (bi == INT_MAX) ? 0 : bi;
+                    }
+                    __syncthreads();
+                    if (warp == 0) {
+                        int x = -1;
+                        bool tok_ok = true;
+                        if (lane < k) {
+                            x = __ldg(p.tokens + static_cast<int64_t>(b) * k + lane);
+                            tok_ok = (x >= 0 && x < p.V);
+                        }
+                        const int bits = (__any_sync(kFull, !tok_ok) ? kStToken : 0) | (nan_sh ? kStLogit : 0);
+                        const unsigned mism = __ballot_sync(kFull, lane < k && x != g_sh[lane < k ? lane : 0]);
+                        const int n = mism ? __ffs(mism) - 1 : k;
+                        int32_t *out = p.out + static_cast<int64_t>(b) * (k + 1);
+                        for (int jj = lane; jj <= k; jj += 32) {
+                            int v = -1;
+                            if (!bits) v = (jj < n) ? x : (jj == n ? g_sh[n] : -1);  // jj < n implies jj == lane
+                            out[jj] = v;
+                        }
+                        if (lane == 0) {
+                            p.acc[b] = bits ? -1 : n;
+                            report(p.status, bits);
+                        }
+                    }
+                }
+                ++rq;
+            }
         }
-        cluster.sync();
-        if (rank == 0) {
-            if (tid == 0) nan_sh = 0;
-            __syncthreads();
-            for (int j = tid; j <= k; j += kThreads) {
-                float bv = -INFINITY;
-                int bi = INT_MAX;
-                bool nan = false;
-                for (int r = 0; r < CL; ++r) {  // slices in index order
-                    const float2 *rp = cluster.map_shared_rank(&part[buf][0], r);
-                    const float2 v = rp[j];
-                    if (v.x != v.x) nan = true;
-                    else argmax_take(bv, bi, v.x, __float_as_int(v.y));
-                }
-                if (nan) atomicOr(&nan_sh, 1);
-                g_sh[j] = (bi == INT_MAX) ? 0 : bi;
-            }
-            __syncthreads();
-            if (warp == 0) {
-                int x = -1;
-                bool tok_ok = true;
-                if (lane < k) {
-                    x = __ldg(p.tokens + static_cast<int64_t>(b) * k + lane);
-                    tok_ok = (x >= 0 && x < p.V);
-                }
-                const int bits = (__any_sync(kFull, !tok_ok) ? kStToken : 0) |
-                                 (nan_sh ? kStLogit : 0);
-                const unsigned mism = __ballot_sync(kFull, lane < k && x != g_sh[lane < k ? lane : 0]);
-                const int n = mism ? __ffs(mism) - 1 : k;
-                int32_t *out = p.out + static_cast<int64_t>(b) * (k + 1);
-                for (int j = lane; j <= k; j += 32) {
-                    int v = -1;
-                    if (!bits) v = (j < n) ? x : (j == n ? g_sh[n] : -1);  // j < n implies j == lane
-                    out[j] = v;
-                }
-                if (lane == 0) {
-                    p.acc[b] = bits ? -1 : n;
-                    report(p.status, bits);
-                }
-            }
-        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) cur[u] = nxt[u];
+        b = nb;
+        j = nj;
+        it = nit;
     }
     cluster.sync();  // no block leaves while rank 0 may still read its partials
 }
