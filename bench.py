@@ -1,7 +1,8 @@
 """Benchmark of the verification sampler (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--config batched|single|greedy|tree|tree-stochastic]
+                    [--config batched|single|greedy|tree|tree-stochastic|
+                              greedy-walk|tree-walk]
 
 A step is one verification call over one batch of synthetic inputs: for the
 default workload, 64 requests x 8 drafts over a 128256-entry bf16
@@ -12,6 +13,11 @@ per second), whole job; achieved HBM GB/s is reported in `roofline`.
 N > 1 (launched by torchrun, one process per GPU): every rank verifies its
 own batch (requests are independent: no collective on the data path); the
 time is the max over ranks of the device-timed region.
+
+The walk configurations time the greedy calls that read only the rows
+their result depends on (spec_verify_greedy_walk, spec_verify_tree_greedy_walk)
+on the greedy and tree workloads; the metric counts the same verify rows as
+the full calls, and `roofline` counts the bytes of the rows actually read.
 
 `--impl reference` times the fp64 CPU oracle on the host, on a bounded
 sample of the same workload (rank 0 only).
@@ -38,7 +44,11 @@ KERNEL_OF = {
     "greedy": "k_greedy_cluster (one launch per call)",
     "tree": "k_pass1 + k_decide (programmatic dependents)",
     "tree-stochastic": "k_pass1 + k_decide + k_pass2 + k_finalize (programmatic dependents)",
+    "greedy-walk": "k_greedy_walk (one launch per call)",
+    "tree-walk": "k_greedy_walk (one launch per call)",
 }
+WALKS = ("greedy-walk", "tree-walk")
+TREES = ("tree", "tree-stochastic", "tree-walk")
 L2_BYTES = 126 * 2 ** 20
 
 
@@ -86,16 +96,43 @@ def make_workload(name, seed):
         return wl.config_batched(seed=seed)
     if name == "single":
         return wl.config_single(seed=seed)
-    if name == "greedy":
+    if name in ("greedy", "greedy-walk"):
         return wl.config_greedy(seed=seed)
-    if name in ("tree", "tree-stochastic"):
+    if name in TREES:
         return wl.config_tree(seed=seed)
     raise ValueError(name)
+
+
+def walk_rows_read(name, w):
+    """Rows a walking greedy call reads: the root and every kept node (a
+    linear chain: rows 0..n of each request).  Counted on the host from the
+    inputs, for the byte count of the roofline."""
+    from speculative_decoding_verification_87_b200.workloads import as_f32
+    am = np.argmax(as_f32(w.target, w.vocab), axis=-1)
+    if name == "greedy-walk":
+        match = (w.tokens == am[:, :-1])
+        n = np.where(match.all(axis=1), w.k, np.argmin(match, axis=1))
+        return int((n + 1).sum())
+    kept = np.zeros(w.parents.shape, bool)
+    kept[:, 0] = True
+    for i in range(1, w.parents.shape[1]):
+        par = w.parents[:, i]
+        rows = np.arange(w.parents.shape[0])
+        kept[:, i] = kept[rows, par] & (w.node_tokens[:, i] == am[rows, par])
+    return int(kept.sum())
 
 
 def workload_facts(name, w):
     """(rows per step, algorithmic bytes per step, config dict)."""
     esz = 2 if w.dtype == "bf16" else 4
+    if name in WALKS:
+        rows, full_bytes, cfg = workload_facts("greedy" if name == "greedy-walk" else "tree", w)
+        read = walk_rows_read(name, w)
+        row_bytes = w.vocab * esz
+        io = full_bytes - rows * row_bytes
+        cfg = dict(cfg, workload=cfg["workload"].replace(" verify", " verify (walk)"),
+                   rows_read_per_step=read, bytes_avoided_per_step=(rows - read) * row_bytes)
+        return rows, read * row_bytes + io, cfg
     if name in ("batched", "single"):
         B, k, V = w.batch, w.k, w.vocab
         rows = B * (k + 1)
@@ -240,6 +277,11 @@ def whole_job_rate(rows_per_step, steps, world, ms_max):
 
 
 # -------------------------------------------------------------- our arm
+def torch_empty_like(t):
+    import torch
+    return torch.empty_like(t)
+
+
 class Runner:
     """Binds one workload's device buffers to the C-ABI call of its mode."""
 
@@ -257,19 +299,33 @@ class Runner:
         self.dev = dev
         self.target = dev(w.target)
         self.draft = dev(w.draft)
-        if name in ("tree", "tree-stochastic"):
+        if name in TREES:
             self.tokens = dev(w.node_tokens)
             self.parents = dev(w.parents)
             W = w.max_depth + 1
             self.out = torch.empty((w.batch, W), dtype=torch.int32, device=device)
-            # pass 1 + decide, then pass 2 + finalize for the stochastic draw
-            self.kernels_per_call = 4 if name == "tree-stochastic" else 2
+            # pass 1 + decide, then pass 2 + finalize for the stochastic draw;
+            # the walk is one kernel
+            self.kernels_per_call = {"tree-stochastic": 4, "tree": 2}.get(name, 1)
         else:
             self.tokens = dev(w.tokens.astype(np.int32))
             self.out = torch.empty((w.batch, w.k + 1), dtype=torch.int32, device=device)
-            # greedy: the cluster kernel; linear stochastic: k_fused
+            # greedy: a cluster kernel; linear stochastic: k_fused
             self.kernels_per_call = 1
         self.acc = torch.empty((w.batch,), dtype=torch.int32, device=device)
+
+    def clone(self):
+        """The same inputs at another device address (a fresh target copy):
+        calls that read few rows cycle over copies so that every call reads
+        HBM, not L2."""
+        import copy
+        c = copy.copy(self)
+        c.target = self.target.clone()
+        if self.name in ("batched", "single", "tree-stochastic"):  # the modes that read drafts
+            c.draft = self.draft.clone()
+        c.out = torch_empty_like(self.out)
+        c.acc = torch_empty_like(self.acc)
+        return c
 
     def call(self, offset, target=None, draft=None, tokens=None):
         b, w = self.binding, self.w
@@ -282,6 +338,12 @@ class Runner:
         elif self.name == "greedy":
             b.spec_verify_greedy(target, tokens, w.vocab, out_tokens=self.out,
                                  accepted_len=self.acc)
+        elif self.name == "greedy-walk":
+            b.spec_verify_greedy_walk(target, tokens, w.vocab, out_tokens=self.out,
+                                      accepted_len=self.acc)
+        elif self.name == "tree-walk":
+            b.spec_verify_tree_greedy_walk(target, tokens, self.parents, w.max_depth, w.vocab,
+                                           out_tokens=self.out, accepted_len=self.acc)
         else:
             b.spec_verify_tree(target, draft, tokens, self.parents, w.max_depth, w.vocab,
                                self.name == "tree-stochastic", w.temperature, 1234, offset,
@@ -298,13 +360,26 @@ def run_ours(args, rank, world, local):
     device = torch.device("cuda", local)
     name = args.config
     sets = [make_workload(name, seed=s) for s in shard_seeds(rank)]
-    rows, alg_bytes, cfg = workload_facts(name, sets[0])
+    facts = [workload_facts(name, w) for w in sets]
+    rows, _, cfg = facts[0]
+    # the walks read a data-dependent number of rows: the mean of the two sets
+    alg_bytes = float(np.mean([f[1] for f in facts]))
+    if name in WALKS:
+        cfg = dict(cfg, rows_read_per_step=float(np.mean([f[2]["rows_read_per_step"] for f in facts])),
+                   bytes_avoided_per_step=float(np.mean([f[2]["bytes_avoided_per_step"]
+                                                         for f in facts])))
     runners = [Runner(name, w, device) for w in sets]
+    # every call must read HBM: the sets (or copies of them) a cycle of calls
+    # reads hold several times the L2
+    n_cycle = max(2, int(np.ceil(4 * L2_BYTES / alg_bytes)))
+    n_cycle += n_cycle % 2
+    while len(runners) < n_cycle:
+        runners.append(runners[len(runners) % 2].clone())
     stream = torch.cuda.current_stream(device)
 
     # warm-up
     for i in range(args.warmup):
-        runners[i % 2].call(offset=i)
+        runners[i % len(runners)].call(offset=i)
     torch.cuda.synchronize(device)
     barrier(world)
 
@@ -316,7 +391,7 @@ def run_ours(args, rank, world, local):
         barrier(world)
         start.record(stream)
         for i in range(args.steps):
-            runners[i % 2].call(offset=args.warmup + i)
+            runners[i % len(runners)].call(offset=args.warmup + i)
         stop.record(stream)
         torch.cuda.synchronize(device)
         barrier(world)
@@ -325,8 +400,8 @@ def run_ours(args, rank, world, local):
     value = whole_job_rate(rows, args.steps, world, ms_max)
     # tokens a call emits (accepted drafts + the drawn token), from each
     # input set's last call
-    acc = np.concatenate([r.acc.cpu().numpy() for r in runners])
-    emitted_per_step = float(np.mean(acc + 1)) * acc.size / len(runners)
+    acc = np.concatenate([r.acc.cpu().numpy() for r in runners[:2]])
+    emitted_per_step = float(np.mean(acc + 1)) * acc.size / 2
     tokens_per_s = whole_job_rate(emitted_per_step, args.steps, world, ms_max)
     step_s = ms_max / 1e3 / args.steps
     peak, peak_src = _peaks()
@@ -352,8 +427,9 @@ def run_ours(args, rank, world, local):
             "dtype": sets[0].dtype,
             "data": "synthetic",
             "config": dict(cfg, parallelism=f"dp{world} (independent request shards)",
-                           l2="inputs larger than L2: 2 resident input sets of "
-                              f"{alg_bytes / 1e6:.1f} MB alternate",
+                           l2=f"inputs larger than L2: calls cycle over {len(runners)} resident "
+                              f"input sets (2 seeds, copies at distinct addresses), "
+                              f"{alg_bytes / 1e6:.1f} MB read per call",
                            requests_per_rank=sets[0].batch),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
@@ -379,7 +455,7 @@ def run_e2e(args, runner, w, device, world):
     import torch
     tgt_h = torch.from_numpy(np.ascontiguousarray(w.target)).pin_memory()
     drf_h = torch.from_numpy(np.ascontiguousarray(w.draft)).pin_memory()
-    tok_src = w.node_tokens if runner.name in ("tree", "tree-stochastic") else w.tokens
+    tok_src = w.node_tokens if runner.name in TREES else w.tokens
     tok_h = torch.from_numpy(np.ascontiguousarray(tok_src.astype(np.int32))).pin_memory()
     if w.target.dtype == np.uint16:
         tgt_h, drf_h = tgt_h.view(torch.bfloat16), drf_h.view(torch.bfloat16)
@@ -388,7 +464,7 @@ def run_e2e(args, runner, w, device, world):
     tok_d = torch.empty(tok_h.shape, dtype=tok_h.dtype, device=device)
     out_h = torch.empty(runner.out.shape, dtype=torch.int32).pin_memory()
     acc_h = torch.empty(runner.acc.shape, dtype=torch.int32).pin_memory()
-    needs_draft = runner.name not in ("greedy", "tree")
+    needs_draft = runner.name in ("batched", "single", "tree-stochastic")
     stream = torch.cuda.current_stream(device)
 
     def step(i):
@@ -442,7 +518,7 @@ def oracle_call(name, s, offset):
     if name in ("batched", "single"):
         oracle.verify_linear(s.target, s.draft, s.tokens, s.vocab, s.temperature, 1234, offset)
         return s.target.shape[0] * s.target.shape[1]
-    if name == "greedy":
+    if name in ("greedy", "greedy-walk"):
         oracle.verify_greedy(s.target, s.tokens, s.vocab)
         return s.target.shape[0] * s.target.shape[1]
     oracle.verify_tree(s.target, s.draft, s.node_tokens, s.parents, s.max_depth, s.vocab,
@@ -530,7 +606,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="batched",
-                    choices=["batched", "single", "greedy", "tree", "tree-stochastic"])
+                    choices=["batched", "single", "greedy", "tree", "tree-stochastic",
+                             "greedy-walk", "tree-walk"])
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -216,6 +216,39 @@ SPECVERIFY_API int spec_verify_tree(const void *target_logits, const void *draft
                      void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Greedy verification that reads only the rows its result depends on.
+ * Same definition and outputs as spec_verify_greedy (greedy) and
+ * spec_verify_tree with stochastic == 0 (tree): "Accelerating Sonar through
+ * speculation", sections "Target-Draft" and "EAGLE" -- a node is kept when
+ * its parent is kept and its token is the argmax of the parent's target row,
+ * and the output is the deepest kept path plus the argmax after it.  Only
+ * the rows of kept nodes (and the root) decide that output, so these calls
+ * walk from the root and read exactly those rows: spec_verify_greedy_walk
+ * reads target rows 0..n of each request (n + 1 of k + 1 rows),
+ * spec_verify_tree_greedy_walk one row per kept node.  Each level costs a
+ * dependent step, so they pay off when few drafts are kept.
+ * Arguments, layouts, limits and outputs are those of spec_verify_greedy and
+ * spec_verify_tree (draft logits, temperature, seed and offset do not
+ * apply; no workspace).  Input errors are reported as there, with one
+ * difference: a NaN logit is detected only in a row the walk reads (a NaN
+ * in a row of a rejected node cannot change the result and is not seen).
+ * Malformed parents, a node deeper than max_depth and out-of-range tokens
+ * are detected for every node, as in the full calls.
+ */
+SPECVERIFY_API int spec_verify_greedy_walk(const void *target_logits, spec_dtype_t dtype,
+                                           int64_t row_stride, const int32_t *draft_tokens,
+                                           int batch, int k, int vocab, int32_t *out_tokens,
+                                           int32_t *accepted_len, int32_t *status,
+                                           cudaStream_t stream);
+
+SPECVERIFY_API int spec_verify_tree_greedy_walk(const void *target_logits, spec_dtype_t dtype,
+                                                int64_t row_stride, const int32_t *node_tokens,
+                                                const int32_t *parents, int batch, int num_nodes,
+                                                int max_depth, int vocab, int32_t *out_tokens,
+                                                int32_t *accepted_len, int32_t *out_path_nodes,
+                                                int32_t *status, cudaStream_t stream);
+
+/*
  * Diagnostic: the uniforms the kernels draw.  out [batch][count] (device,
  * double) = U(seed, b, first_position + i, purpose, offset).  Lets a caller
  * check the device Philox stream against an independent implementation.

@@ -23,7 +23,8 @@ STATUS_TOKEN, STATUS_TREE, STATUS_LOGIT, STATUS_TIMEOUT = 1, 2, 4, 8
 MAX_K, MAX_NODES = 32, 1024
 SYMBOLS = ("spec_verify_workspace_size", "spec_verify_strerror", "spec_verify_linear",
            "spec_verify_greedy", "spec_verify_tree", "spec_verify_debug_uniforms",
-           "spec_verify_linear_noalloc", "spec_verify_debug_exp2")
+           "spec_verify_linear_noalloc", "spec_verify_debug_exp2", "spec_verify_greedy_walk",
+           "spec_verify_tree_greedy_walk")
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 _lib = None
@@ -67,6 +68,11 @@ def load_library(path: str = LIB_PATH):
         L.spec_verify_linear_noalloc.argtypes = [_P, _P, _I, _I64, _P, _I, _I, _I, _F, _U64, _U32,
                                                  _P, _P, _P, _P, _P, _P]
         L.spec_verify_linear_noalloc.restype = _I
+        L.spec_verify_greedy_walk.argtypes = [_P, _I, _I64, _P, _I, _I, _I, _P, _P, _P, _P]
+        L.spec_verify_greedy_walk.restype = _I
+        L.spec_verify_tree_greedy_walk.argtypes = [_P, _I, _I64, _P, _P, _I, _I, _I, _I, _P, _P,
+                                                   _P, _P, _P]
+        L.spec_verify_tree_greedy_walk.restype = _I
         L.spec_verify_debug_exp2.argtypes = [_P, _P, _I, _I, _P]
         L.spec_verify_debug_exp2.restype = _I
         _lib = L
@@ -183,6 +189,59 @@ def spec_verify_greedy(target_logits, draft_tokens, vocab, out_tokens=None, acce
         _ptr(out_tokens), _ptr(accepted_len), _ptr(status), _stream(stream))
     _check(rc, "spec_verify_greedy")
     return out_tokens, accepted_len
+
+
+def spec_verify_greedy_walk(target_logits, draft_tokens, vocab, out_tokens=None,
+                            accepted_len=None, status=None, stream=None):
+    """As spec_verify_greedy, reading only target rows 0..n of each request."""
+    _need_cuda("target_logits", target_logits)
+    B, R, stride = target_logits.shape
+    k = R - 1
+    _need_cuda("draft_tokens", draft_tokens, torch.int32, (B, k))
+    dev = target_logits.device
+    if out_tokens is None:
+        out_tokens = torch.empty((B, k + 1), dtype=torch.int32, device=dev)
+    if accepted_len is None:
+        accepted_len = torch.empty((B,), dtype=torch.int32, device=dev)
+    _need_cuda("out_tokens", out_tokens, torch.int32, (B, k + 1))
+    _need_cuda("accepted_len", accepted_len, torch.int32, (B,))
+    if status is not None:
+        _need_cuda("status", status, torch.int32)
+    rc = load_library().spec_verify_greedy_walk(
+        _ptr(target_logits), _dtype_code(target_logits), stride, _ptr(draft_tokens), B, k, vocab,
+        _ptr(out_tokens), _ptr(accepted_len), _ptr(status), _stream(stream))
+    _check(rc, "spec_verify_greedy_walk")
+    return out_tokens, accepted_len
+
+
+def spec_verify_tree_greedy_walk(target_logits, node_tokens, parents, max_depth, vocab,
+                                 out_tokens=None, accepted_len=None, out_path_nodes=None,
+                                 status=None, stream=None):
+    """As spec_verify_tree with stochastic=False, reading only the rows of
+    kept nodes.  Returns (out_tokens [B][D+1], accepted_len [B],
+    out_path_nodes [B][D+1] or None)."""
+    _need_cuda("target_logits", target_logits)
+    B, N, stride = target_logits.shape
+    _need_cuda("node_tokens", node_tokens, torch.int32, (B, N))
+    _need_cuda("parents", parents, torch.int32, (B, N))
+    dev = target_logits.device
+    W = max_depth + 1
+    if out_tokens is None:
+        out_tokens = torch.empty((B, W), dtype=torch.int32, device=dev)
+    if accepted_len is None:
+        accepted_len = torch.empty((B,), dtype=torch.int32, device=dev)
+    _need_cuda("out_tokens", out_tokens, torch.int32, (B, W))
+    _need_cuda("accepted_len", accepted_len, torch.int32, (B,))
+    if out_path_nodes is not None:
+        _need_cuda("out_path_nodes", out_path_nodes, torch.int32, (B, W))
+    if status is not None:
+        _need_cuda("status", status, torch.int32)
+    rc = load_library().spec_verify_tree_greedy_walk(
+        _ptr(target_logits), _dtype_code(target_logits), stride, _ptr(node_tokens),
+        _ptr(parents), B, N, max_depth, vocab, _ptr(out_tokens), _ptr(accepted_len),
+        _ptr(out_path_nodes), _ptr(status), _stream(stream))
+    _check(rc, "spec_verify_tree_greedy_walk")
+    return out_tokens, accepted_len, out_path_nodes
 
 
 def spec_verify_tree(target_logits, draft_logits, node_tokens, parents, max_depth, vocab,

@@ -108,3 +108,28 @@ def test_greedy_and_tree_host_validation(lib):
     assert t(temp=-1.0) == SPEC_EINVAL
     assert t(ws_bytes=8) == SPEC_EWORKSPACE
     assert t(batch=0) == SPEC_OK
+
+
+def test_walk_host_validation(lib):
+    P = ctypes.c_void_p
+    g = lambda **kw: lib.spec_verify_greedy_walk(P(kw.get("tl", 0x1000)), kw.get("dtype", 0),
+                                                 kw.get("stride", 64), P(kw.get("tok", 0x2000)),
+                                                 kw.get("batch", 3), kw.get("k", 2),
+                                                 kw.get("vocab", 50), P(0x3000), P(0x4000), None,
+                                                 None)
+    assert g(k=0) == SPEC_EINVAL and g(k=33) == SPEC_EUNSUPPORTED
+    assert g(batch=-1) == SPEC_EINVAL
+    assert g(stride=63) == SPEC_EALIGN and g(vocab=65) == SPEC_EINVAL and g(vocab=0) == SPEC_EINVAL
+    assert g(tl=0x1004) == SPEC_EALIGN and g(tl=0) == SPEC_EINVAL and g(tok=0) == SPEC_EINVAL
+    assert g(dtype=3) == SPEC_EINVAL
+    assert g(batch=0) == SPEC_OK and g(batch=0, tl=0, tok=0) == SPEC_OK
+
+    def t(**kw):
+        return lib.spec_verify_tree_greedy_walk(P(kw.get("tl", 0x1000)), 1, 64, P(0x3000),
+                                                P(kw.get("par", 0x3800)), kw.get("batch", 2),
+                                                kw.get("nodes", 60), kw.get("depth", 6), 60,
+                                                P(0x4000), P(0x5000), None, None, None)
+    assert t(nodes=0) == SPEC_EINVAL and t(nodes=1025) == SPEC_EUNSUPPORTED
+    assert t(depth=0) == SPEC_EINVAL and t(batch=-2) == SPEC_EINVAL
+    assert t(par=0) == SPEC_EINVAL and t(tl=0x1002) == SPEC_EALIGN
+    assert t(batch=0) == SPEC_OK and t(batch=0, tl=0, par=0) == SPEC_OK
