@@ -172,7 +172,7 @@ def test_tree_walk_shared_sibling_tokens(sv, orc, B, N, max_depth, V, dtype):
 
 
 def test_tree_walk_1024_node_chain_kept_to_the_end(sv, orc):
-    B, N, V = 2, 1024, 37
+    B, N, V = 2, 1024, 36  # fp32 rows of 144 bytes (a multiple of 16)
     t = np.zeros((B, N, V), np.float32)
     t[:, :, 11] = 1.0
     parents = np.tile(np.arange(-1, N - 1, dtype=np.int32), (B, 1))
@@ -195,7 +195,7 @@ def test_chain_tree_walk_equals_linear_walk(sv):
 
 def test_tree_walk_errors(sv, orc):
     rng = np.random.default_rng(5)
-    B, N, V = 8, 12, 7
+    B, N, V = 8, 12, 8  # fp32 rows of 32 bytes
     t, tokens, _ = random_tree(rng, B, N, 4, V, keep=1.0)
     parents = np.tile(np.array([-1, 0, 0, 1, 1, 2, 3, 4, 5, 6, 7, 8], np.int32), (B, 1))
     am = np.argmax(t, axis=-1)
