@@ -15,10 +15,12 @@
 // of each row to (max, lowest argmax, NaN seen) and, after one cluster
 // barrier, every block merges all CL partials through distributed shared
 // memory.  All blocks keep identical copies of the queue and request state:
-// every update is computed from the same inputs in the same order, so no
+// every update is computed from the same inputs, and where several threads
+// update one record they do it with order-free atomics (OR, max), so no
 // second barrier is needed to broadcast it.  The children of a processed
 // node whose token equals the row's argmax join the queue; a request is
 // done when none of its rows is pending, and rank 0 writes its outputs.
+// The bookkeeping between rounds is one warp wide (a lane per request slot).
 //
 // Node records (parent, token, depth) of the requests in flight are cached
 // in shared memory when a request is admitted; depths come from pointer
@@ -34,70 +36,115 @@
 namespace sv {
 
 constexpr int kWalkRows = 16;    // rows reduced per round (one cluster barrier)
-constexpr int kWalkSlots = 32;   // requests in flight per cluster
+constexpr int kWalkSlots = 32;   // requests in flight per cluster (one warp's lanes)
 constexpr int kWalkCache = 2048; // cached node records per block (A * N <= this)
 constexpr int kWalkRing = 2048;  // pending rows; a power of two >= kWalkCache
 constexpr int kWalkJumps = 12;   // pointer-jumping rounds (2^11 > SPEC_MAX_NODES)
 static_assert((kWalkRing & (kWalkRing - 1)) == 0 && kWalkRing >= kWalkCache, "ring size");
 static_assert(kWalkCache % kThreads == 0, "cache is scanned in whole block strides");
+static_assert(kWalkSlots == 32 && kWalkRows <= 32, "slots and rows are warp lanes");
 
 struct WalkShared {
     float2 part[2][kWalkRows];         // this block's (max or NaN, argmax bits) per row
     float redf[kWarps];
     int redi[kWarps];
     int g[kWalkRows];                  // merged argmax of the round's rows
-    int nan[kWalkRows];                // a NaN was seen in the row
     int cnt[kWalkRows];                // children queued by the row
     unsigned ring[kWalkRing];          // pending rows: node | slot << 16
     int tok[kWalkCache];               // node token, at slot * N + node
     short par[kWalkCache];             // node parent (-1 for the root)
     short dep[kWalkCache];             // node depth
     short anc[kWalkCache];             // pointer-jumping scratch
+    // deepest kept node of the slot's request, as one key whose maximum is
+    // the deepest node with the lowest index: depth << 42 | (1023 - node) << 32 | argmax
+    unsigned long long best[kWalkSlots];
     int req[kWalkSlots];               // request of the slot, -1 when free
     int pend[kWalkSlots];              // rows of the slot queued or in the round
     int err[kWalkSlots];               // status bits of the request
-    int bd[kWalkSlots], bn[kWalkSlots], bg[kWalkSlots];  // deepest kept node: depth, index, argmax
-    int fresh[kWalkSlots];             // admitted by the current admission pass
-    int qh, qt, next, active, any_fresh;
+    int fresh[kWalkSlots];             // slots filled by the last admission, in slot order
+    int qh, qt, next, active, nfresh;
 };
 
-// Fill free slots with the cluster's next requests and cache their node
-// records; requests with malformed input get their error bits here (and no
-// queued row); the others queue their root.
-__device__ __forceinline__ void walk_admit(const Params &p, WalkShared &sh, int A, int ncl,
-                                           bool chain)
+// Warp 0: requests with no pending row are done (rank 0 writes their
+// outputs) and their slots are freed; free slots then take the cluster's
+// next requests in slot order.  One lane per slot.
+__device__ __forceinline__ void walk_book(const Params &p, WalkShared &sh, int A, int ncl, int rank)
 {
-    const int tid = threadIdx.x;
-    const int N = p.N;
-    if (tid == 0) {
-        int any = 0;
-        for (int s = 0; s < A; ++s) {
-            sh.fresh[s] = 0;
-            if (sh.req[s] < 0 && sh.next < p.B) {
-                sh.req[s] = sh.next;
-                sh.next += ncl;
-                sh.fresh[s] = 1;
-                sh.err[s] = 0;
-                sh.pend[s] = 0;
-                sh.bd[s] = -1;
-                sh.bn[s] = 0;
-                sh.bg[s] = 0;
-                ++sh.active;
-                any = 1;
+    const int lane = threadIdx.x & 31;
+    const int N = p.N, W = p.max_depth + 1;
+    const unsigned lt = (1u << lane) - 1u;
+    const bool in = lane < A;
+    const int rq = in ? sh.req[lane] : -1;
+    const bool done = in && rq >= 0 && sh.pend[lane] == 0;
+    const unsigned dmask = __ballot_sync(kFull, done);
+    if (rank == 0) {
+        for (unsigned m = dmask; m; m &= m - 1u) {
+            const int t = __ffs(m) - 1;
+            const int b = __shfl_sync(kFull, rq, t);
+            const int err = sh.err[t];
+            const unsigned long long key = sh.best[t];
+            const int D = err ? -1 : static_cast<int>(key >> 42);
+            int32_t *out = p.out + static_cast<int64_t>(b) * W;
+            int32_t *path = p.path ? p.path + static_cast<int64_t>(b) * W : nullptr;
+            for (int j = D + 1 + lane; j < W; j += 32) {  // past the bonus (everything on an error)
+                out[j] = -1;
+                if (path) path[j] = -1;
+            }
+            if (lane == 0) {
+                if (err) {
+                    p.acc[b] = -1;
+                    report(p.status, err);
+                } else {
+                    const int base = t * N;
+                    for (int node = 1023 - static_cast<int>((key >> 32) & 1023u); node > 0;
+                         node = sh.par[base + node]) {
+                        const int d = sh.dep[base + node];
+                        out[d - 1] = sh.tok[base + node];
+                        if (path) path[d] = node;
+                    }
+                    if (path) path[0] = 0;
+                    out[D] = static_cast<int>(static_cast<unsigned>(key & 0xFFFFFFFFull));
+                    p.acc[b] = D;
+                }
             }
         }
-        sh.any_fresh = any;
     }
-    __syncthreads();
-    if (!sh.any_fresh) return;  // block-uniform
+    const int next = sh.next;
+    const bool free_slot = in && (rq < 0 || done);
+    const unsigned fmask = __ballot_sync(kFull, free_slot);
+    const int nr = next + __popc(fmask & lt) * ncl;
+    const bool fresh = free_slot && nr < p.B;
+    const unsigned frmask = __ballot_sync(kFull, fresh);
+    if (done) sh.req[lane] = -1;
+    if (fresh) {
+        sh.req[lane] = nr;
+        sh.pend[lane] = 0;
+        sh.err[lane] = 0;
+        sh.best[lane] = 0ull;
+        sh.fresh[__popc(frmask & lt)] = lane;
+    }
+    __syncwarp();
+    if (lane == 0) {
+        const int nf = __popc(frmask);
+        sh.next = next + nf * ncl;
+        sh.active += nf - __popc(dmask);
+        sh.nfresh = nf;
+    }
+}
 
-    // node records of the fresh slots (a chain's are implicit but cached alike)
-    for (int e = tid; e < A * N; e += kThreads) {
-        const int s = e / N, i = e - s * N;
-        if (!sh.fresh[s]) continue;
+// Whole block, after an admission: cache the node records of the fresh
+// requests, find malformed input (its error bits, and no queued row), and
+// queue the roots of the others.
+__device__ __forceinline__ void walk_load(const Params &p, WalkShared &sh, bool chain)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int N = p.N, E = sh.nfresh * N;
+    for (int x = tid; x < E; x += kThreads) {
+        const int f = x / N, i = x - f * N;
+        const int s = sh.fresh[f], e = s * N + i;
         const int b = sh.req[s];
         int par = i - 1, tk = 0, bits = 0;
-        if (chain) {
+        if (chain) {  // the chain of a linear request: parent i - 1, token = draft i - 1
             if (i > 0) {
                 tk = __ldg(p.tokens + static_cast<int64_t>(b) * p.k + (i - 1));
                 if (tk < 0 || tk >= p.V) bits |= kStToken;
@@ -122,25 +169,30 @@ __device__ __forceinline__ void walk_admit(const Params &p, WalkShared &sh, int 
     }
     __syncthreads();
 
-    // depths: dep[e] is the distance from node e to anc[e]; each round
-    // doubles the jump, and a node whose jump reached the root is final
+    // depths by pointer jumping: dep[e] is the distance from node e to
+    // anc[e]; each round doubles the jump, and a jump that reached the root
+    // is final
     if (!chain) {
         constexpr int kPer = kWalkCache / kThreads;
+        auto entry = [&](int x) {
+            const int f = x / N;
+            return sh.fresh[f] * N + (x - f * N);
+        };
 #pragma unroll 1
         for (int round = 0; round < kWalkJumps; ++round) {
             short nd[kPer], na[kPer];
             int more = 0;
 #pragma unroll
             for (int j = 0; j < kPer; ++j) {
-                const int e = tid + j * kThreads;
+                const int x = tid + j * kThreads;
                 nd[j] = na[j] = 0;
-                if (e < A * N) {
-                    const int s = e / N;
+                if (x < E) {
+                    const int e = entry(x);
                     const int a = sh.anc[e];
                     nd[j] = sh.dep[e];
                     na[j] = static_cast<short>(a);
-                    if (sh.fresh[s] && a != 0) {
-                        const int base = s * N;
+                    if (a != 0) {
+                        const int base = e - (x % N);
                         nd[j] = static_cast<short>(nd[j] + sh.dep[base + a]);
                         na[j] = sh.anc[base + a];
                         more |= (na[j] != 0);
@@ -150,8 +202,9 @@ __device__ __forceinline__ void walk_admit(const Params &p, WalkShared &sh, int 
             __syncthreads();
 #pragma unroll
             for (int j = 0; j < kPer; ++j) {
-                const int e = tid + j * kThreads;
-                if (e < A * N) {
+                const int x = tid + j * kThreads;
+                if (x < E) {
+                    const int e = entry(x);
                     sh.dep[e] = nd[j];
                     sh.anc[e] = na[j];
                 }
@@ -160,70 +213,24 @@ __device__ __forceinline__ void walk_admit(const Params &p, WalkShared &sh, int 
         }
         // a node deeper than max_depth is a malformed tree (checked only
         // when the parent array itself is well formed)
-        for (int e = tid; e < A * N; e += kThreads) {
-            const int s = e / N;
-            if (sh.fresh[s] && !(sh.err[s] & kStTree) && sh.dep[e] > p.max_depth)
-                atomicOr(&sh.err[s], kStTree);
+        for (int x = tid; x < E; x += kThreads) {
+            const int e = entry(x), s = sh.fresh[x / N];
+            if (!(sh.err[s] & kStTree) && sh.dep[e] > p.max_depth) atomicOr(&sh.err[s], kStTree);
         }
         __syncthreads();
     }
-    if (tid == 0) {
-        for (int s = 0; s < A; ++s) {
-            if (sh.fresh[s] && !sh.err[s]) {
-                sh.ring[sh.qt & (kWalkRing - 1)] = static_cast<unsigned>(s) << 16;  // the root
-                ++sh.qt;
-                sh.pend[s] = 1;
-            }
+    if (warp == 0) {
+        const int F = sh.nfresh;
+        const int s = lane < F ? sh.fresh[lane] : 0;
+        const bool ok = lane < F && sh.err[s] == 0;
+        const unsigned m = __ballot_sync(kFull, ok);
+        const int qt = sh.qt;
+        if (ok) {
+            sh.ring[(qt + __popc(m & ((1u << lane) - 1u))) & (kWalkRing - 1)] = static_cast<unsigned>(s) << 16;
+            sh.pend[s] = 1;
         }
-    }
-    __syncthreads();
-}
-
-// Requests with no pending row are done: rank 0 writes their outputs, every
-// block frees their slots.
-__device__ __forceinline__ void walk_complete(const Params &p, WalkShared &sh, int A, int rank)
-{
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int N = p.N, W = p.max_depth + 1;
-    if (rank == 0) {
-        for (int s = warp; s < A; s += kWarps) {
-            if (sh.req[s] < 0 || sh.pend[s] != 0) continue;
-            const int b = sh.req[s];
-            const int err = sh.err[s];
-            const int D = err ? -1 : sh.bd[s];
-            int32_t *out = p.out + static_cast<int64_t>(b) * W;
-            int32_t *path = p.path ? p.path + static_cast<int64_t>(b) * W : nullptr;
-            // entries past the bonus (all of them on an error)
-            for (int j = D + 1 + lane; j < W; j += 32) {
-                out[j] = -1;
-                if (path) path[j] = -1;
-            }
-            if (lane == 0) {
-                if (err) {
-                    p.acc[b] = -1;
-                    report(p.status, err);
-                } else {
-                    const int base = s * N;
-                    for (int node = sh.bn[s]; node > 0; node = sh.par[base + node]) {
-                        const int d = sh.dep[base + node];
-                        out[d - 1] = sh.tok[base + node];
-                        if (path) path[d] = node;
-                    }
-                    if (path) path[0] = 0;
-                    out[D] = sh.bg[s];
-                    p.acc[b] = D;
-                }
-            }
-        }
-    }
-    __syncthreads();
-    if (tid == 0) {
-        for (int s = 0; s < A; ++s) {
-            if (sh.req[s] >= 0 && sh.pend[s] == 0) {
-                sh.req[s] = -1;
-                --sh.active;
-            }
-        }
+        __syncwarp();
+        if (lane == 0) sh.qt = qt + __popc(m);
     }
     __syncthreads();
 }
@@ -248,7 +255,10 @@ __global__ void __launch_bounds__(kThreads) k_greedy_walk(const Params p, int sl
     const int s_begin = min(p.V, rank * slice), s_end = min(p.V, s_begin + slice);
     const int iters = max(1, (s_end - s_begin + kChunk - 1) / kChunk);
 
-    for (int s = tid; s < kWalkSlots; s += kThreads) sh.req[s] = -1;
+    for (int s = tid; s < kWalkSlots; s += kThreads) {
+        sh.req[s] = -1;
+        sh.pend[s] = 0;
+    }
     if (tid == 0) {
         sh.qh = sh.qt = 0;
         sh.next = cid;
@@ -256,9 +266,14 @@ __global__ void __launch_bounds__(kThreads) k_greedy_walk(const Params p, int sl
     }
     __syncthreads();
 
-    auto row_of = [&](int qh, int r) {
+    auto slot_node = [&](int qh, int r, int &s) {
         const unsigned e = sh.ring[(qh + r) & (kWalkRing - 1)];
-        const int node = static_cast<int>(e & 0xFFFFu), s = static_cast<int>(e >> 16);
+        s = static_cast<int>(e >> 16);
+        return static_cast<int>(e & 0xFFFFu);
+    };
+    auto row_of = [&](int qh, int r) {
+        int s;
+        const int node = slot_node(qh, r, s);
         return static_cast<const char *>(p.tl) +
                (static_cast<int64_t>(sh.req[s]) * N + node) * p.stride * kEsz;
     };
@@ -273,9 +288,9 @@ __global__ void __launch_bounds__(kThreads) k_greedy_walk(const Params p, int sl
         }
     };
 
-    // every iteration admits requests or reduces at least one row, so the
-    // loop ends within (requests owned) * (N + 1) + 2 iterations; the bound
-    // guards the cluster barriers against a logic error
+    // every iteration admits or completes requests or reduces at least one
+    // row, so the loop ends within (requests owned) * (N + 1) + 2
+    // iterations; the bound guards the cluster barriers against a logic error
     const int owned = cid < p.B ? (p.B - cid + ncl - 1) / ncl : 0;
     const int64_t limit = static_cast<int64_t>(owned) * (N + 1) + 4;
     int64_t iter = 0;
@@ -286,11 +301,12 @@ __global__ void __launch_bounds__(kThreads) k_greedy_walk(const Params p, int sl
             if (rank == 0 && tid == 0) report(p.status, kStTimeout);
             break;
         }
-        walk_admit(p, sh, A, ncl, chain);
-        walk_complete(p, sh, A, rank);  // requests rejected at admission
+        if (warp == 0) walk_book(p, sh, A, ncl, rank);
+        __syncthreads();
+        if (sh.nfresh) walk_load(p, sh, chain);
         const int qh = sh.qh, qt = sh.qt;
         const bool done = sh.active == 0 && sh.next >= p.B;
-        __syncthreads();  // all threads hold the control state before thread 0 changes it
+        __syncthreads();  // all threads hold the control state before it changes
         if (done) break;
         if (qh == qt) continue;
         const int nb = min(kWalkRows, qt - qh);
@@ -364,8 +380,8 @@ __global__ void __launch_bounds__(kThreads) k_greedy_walk(const Params p, int sl
         }
         cluster.sync();  // every block's partials of the round are visible
 
-        // merge: CL lanes per row, in slice order (the argmax rule does not
-        // depend on the order)
+        // merge: CL lanes per row (the argmax rule does not depend on the
+        // order); the row's lead lane records errors and the deepest node
         if (tid < kWalkRows * CL) {
             const int r = tid / CL, rr = tid % CL;
             float bv = -INFINITY;
@@ -386,24 +402,15 @@ __global__ void __launch_bounds__(kThreads) k_greedy_walk(const Params p, int sl
                 argmax_take(bv, bi, ov, oi);
             }
             if (rr == 0 && r < nb) {
-                sh.g[r] = (bi == INT_MAX) ? 0 : bi;  // an all -inf row has argmax 0
-                sh.nan[r] = nn;
-            }
-        }
-        __syncthreads();
-
-        // errors and the deepest kept node, in queue order
-        if (tid == 0) {
-            for (int r = 0; r < nb; ++r) {
-                const unsigned e = sh.ring[(qh + r) & (kWalkRing - 1)];
-                const int node = static_cast<int>(e & 0xFFFFu), s = static_cast<int>(e >> 16);
-                if (sh.nan[r]) sh.err[s] |= kStLogit;
-                const int d = sh.dep[s * N + node];
-                if (d > sh.bd[s] || (d == sh.bd[s] && node < sh.bn[s])) {
-                    sh.bd[s] = d;
-                    sh.bn[s] = node;
-                    sh.bg[s] = sh.g[r];
-                }
+                const int g = (bi == INT_MAX) ? 0 : bi;  // an all -inf row has argmax 0
+                sh.g[r] = g;
+                int s;
+                const int node = slot_node(qh, r, s);
+                if (nn) atomicOr(&sh.err[s], kStLogit);
+                const unsigned long long key =
+                    (static_cast<unsigned long long>(sh.dep[s * N + node]) << 42) |
+                    (static_cast<unsigned long long>(1023 - node) << 32) | static_cast<unsigned>(g);
+                atomicMax(&sh.best[s], key);
             }
         }
         __syncthreads();
@@ -412,14 +419,13 @@ __global__ void __launch_bounds__(kThreads) k_greedy_walk(const Params p, int sl
         // per row counts them, then writes them at its prefix offset
         for (int pass = 0; pass < 2; ++pass) {
             for (int r = warp; r < nb; r += kWarps) {
-                const unsigned e = sh.ring[(qh + r) & (kWalkRing - 1)];
-                const int node = static_cast<int>(e & 0xFFFFu), s = static_cast<int>(e >> 16);
+                int s;
+                const int node = slot_node(qh, r, s);
                 const int base = s * N, g = sh.g[r];
                 const bool live = sh.err[s] == 0;
                 int off = qt;
                 if (pass == 1) {
-                    const int c = lane < r ? sh.cnt[lane] : 0;  // r < kWalkRows <= 32
-                    int sum = c;
+                    int sum = lane < r ? sh.cnt[lane] : 0;
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);
                     off += sum;
@@ -434,22 +440,19 @@ __global__ void __launch_bounds__(kThreads) k_greedy_walk(const Params p, int sl
                             static_cast<unsigned>(c) | (static_cast<unsigned>(s) << 16);
                     count += __popc(m);
                 }
-                if (pass == 0 && lane == 0) sh.cnt[r] = count;
+                if (lane == 0) {
+                    if (pass == 0) sh.cnt[r] = count;
+                    else atomicAdd(&sh.pend[s], count - 1);  // the row is done, its children pending
+                }
+            }
+            if (pass == 1 && tid == 0) {
+                int total = 0;
+                for (int r = 0; r < nb; ++r) total += sh.cnt[r];
+                sh.qh = qh + nb;
+                sh.qt = qt + total;
             }
             __syncthreads();
         }
-        if (tid == 0) {
-            int total = 0;
-            for (int r = 0; r < nb; ++r) {
-                const int s = static_cast<int>(sh.ring[(qh + r) & (kWalkRing - 1)] >> 16);
-                sh.pend[s] += sh.cnt[r] - 1;
-                total += sh.cnt[r];
-            }
-            sh.qh = qh + nb;
-            sh.qt = qt + total;
-        }
-        __syncthreads();
-        walk_complete(p, sh, A, rank);
         buf ^= 1;
     }
     cluster.sync();  // no block leaves while another may still read its partials
