@@ -52,29 +52,49 @@ TREES = ("tree", "tree-stochastic", "tree-walk")
 L2_BYTES = 126 * 2 ** 20
 
 
-def csrc_digest():
-    """sha256 over the CUDA sources (sorted by name): identifies the kernels."""
+CSRC = os.path.join(ROOT, "speculative_decoding_verification_87_b200", "csrc")
+
+
+def tu_files(main):
+    """The CUDA sources of one translation unit of the library: the .cu file
+    and the csrc headers it includes, recursively."""
+    import re
+    seen, todo = set(), [main]
+    while todo:
+        name = todo.pop()
+        if name in seen:
+            continue
+        seen.add(name)
+        with open(os.path.join(CSRC, name)) as f:
+            for inc in re.findall(r'^\s*#include\s+"([^"/]+)"', f.read(), re.M):
+                if os.path.exists(os.path.join(CSRC, inc)):
+                    todo.append(inc)
+    return sorted(seen)
+
+
+def tu_digest(main):
+    """sha256 over a translation unit's sources (sorted by name): identifies
+    the kernels it builds and their launches.  The public header holds only
+    declarations and error codes and is not part of it."""
     import hashlib
-    d = os.path.join(ROOT, "speculative_decoding_verification_87_b200", "csrc")
     h = hashlib.sha256()
-    for name in sorted(os.listdir(d)):
-        if name.endswith((".cu", ".cuh")):
-            h.update(name.encode())
-            with open(os.path.join(d, name), "rb") as f:
-                h.update(f.read())
+    for name in tu_files(main):
+        h.update(name.encode())
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()
 
 
 def measured_traffic(workload):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
-    summary (profiles/traffic.json), or None when the kernels have changed
-    since those counters were taken."""
+    summary (profiles/traffic.json), or None when the sources of the kernel's
+    translation unit have changed since those counters were taken."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             entry = json.load(f).get(workload)
     except Exception:
         return None, None
-    if not entry or entry.get("csrc_sha256") != csrc_digest():
+    if not entry or entry.get("tu_sha256") != tu_digest(entry.get("tu", "specverify.cu")):
         return None, None
     return entry["dram_read_bytes"] + entry["dram_write_bytes"], entry.get("summary")
 

@@ -2,8 +2,9 @@
 
     python -m speculative_decoding_verification_87_b200.build [--force]
 
-The library is built from csrc/*.cu (specverify.cu with its headers, and
-noalloc.cu), compiled for sm_100a only, with static cudart and -lineinfo.
+The library is built from csrc/*.cu (specverify.cu with its headers,
+noalloc.cu, and walk.cu with sv_walk.cuh), compiled for sm_100a only,
+with static cudart and -lineinfo.
 """
 import glob
 import os
