@@ -1,0 +1,67 @@
+"""Host-side bookkeeping of bench.py (no GPU): the rows a walking greedy call
+reads, the byte counts built on them, and the translation units that key
+the ncu traffic records."""
+import os
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from speculative_decoding_verification_87_b200 import workloads as wl  # noqa: E402
+
+
+def test_chain_rows_read_match_oracle_accept_lengths(orc):
+    # a linear walk reads rows 0..n of each request: sum(n + 1)
+    for seed in range(3):
+        w = wl.greedy_linear(seed=seed, batch=24, k=5, vocab=300)
+        o = orc.verify_greedy(w.target, w.tokens, w.vocab)
+        assert bench.walk_rows_read("greedy-walk", w) == int((o["acc"] + 1).sum())
+
+
+def test_tree_rows_read_on_a_hand_built_tree():
+    # root 0 with children 1, 2 (same token), 1 -> 3, 2 -> 4; argmax of every
+    # row is token 5, except node 1's row (token 6)
+    V = 8
+    t = np.zeros((1, 5, V), np.float32)
+    t[0, :, 5] = 1.0
+    t[0, 1, 5], t[0, 1, 6] = 0.0, 1.0
+    parents = np.array([[-1, 0, 0, 1, 2]], np.int32)
+    tokens = np.array([[-1, 5, 5, 5, 5]], np.int32)
+    w = wl.TreeWorkload("hand", t, t, tokens, parents, 2, V, 1.0, "f32")
+    # kept: root, 1 and 2 (both match the root's argmax), 4 (matches node 2's
+    # argmax); node 3 does not match node 1's argmax
+    assert bench.walk_rows_read("tree-walk", w) == 4
+
+
+def test_tree_rows_read_bounds_and_chain_equivalence(orc):
+    w = wl.draft_tree(seed=1, batch=4, vocab=500, level_widths=(1, 3, 3, 2))
+    o = orc.verify_tree(w.target, None, w.node_tokens, w.parents, w.max_depth, w.vocab, False,
+                        1.0, 0, 0)
+    read = bench.walk_rows_read("tree-walk", w)
+    # every node on each chosen path is kept, and no more than all nodes
+    assert int((o["acc"] + 1).sum()) <= read <= w.batch * w.num_nodes
+    lin = wl.greedy_linear(seed=4, batch=10, k=3, vocab=200)
+    c = wl.chain_tree_from_linear(lin)
+    assert bench.walk_rows_read("tree-walk", c) == bench.walk_rows_read("greedy-walk", lin)
+
+
+def test_walk_bytes_are_the_rows_read():
+    w = wl.greedy_linear(seed=2, batch=16, k=4, vocab=1000)
+    rows, full, _ = bench.workload_facts("greedy", w)
+    rows_w, walk, cfg = bench.workload_facts("greedy-walk", w)
+    read = bench.walk_rows_read("greedy-walk", w)
+    assert rows_w == rows == 16 * 5
+    assert cfg["rows_read_per_step"] == read
+    assert full - walk == (rows - read) * 1000 * 2 == cfg["bytes_avoided_per_step"]
+    assert "(walk)" in cfg["workload"]
+
+
+def test_translation_units():
+    main = bench.tu_files("specverify.cu")
+    assert {"specverify.cu", "sv_common.cuh", "sv_fused.cuh", "sv_verify.cuh"} <= set(main)
+    assert "sv_walk.cuh" not in main and "walk.cu" not in main
+    assert bench.tu_files("walk.cu") == ["sv_common.cuh", "sv_walk.cuh", "walk.cu"]
+    assert bench.tu_digest("walk.cu") != bench.tu_digest("specverify.cu")
