@@ -291,6 +291,19 @@ def shard_seeds(rank, nsets=2):
     return [1000 * rank + s for s in range(nsets)]
 
 
+def empirical_alpha(acc, k):
+    """Per-position acceptance rate of linear verification: alpha_j =
+    #(n > j) / #(n >= j) over the requests (n < 0, an input error, is left
+    out); None where no request reached position j."""
+    a = np.asarray(acc)
+    a = a[a >= 0]
+    out = []
+    for j in range(k):
+        reach = int((a >= j).sum())
+        out.append(float((a > j).sum()) / reach if reach else None)
+    return out
+
+
 def whole_job_rate(rows_per_step, steps, world, ms_max):
     """Rows per second of the whole job: every rank's rows over the slowest rank's time."""
     return rows_per_step * steps * world / (ms_max / 1e3)
@@ -423,6 +436,8 @@ def run_ours(args, rank, world, local):
     acc = np.concatenate([r.acc.cpu().numpy() for r in runners[:2]])
     emitted_per_step = float(np.mean(acc + 1)) * acc.size / 2
     tokens_per_s = whole_job_rate(emitted_per_step, args.steps, world, ms_max)
+    requests_per_s = whole_job_rate(sets[0].batch, args.steps, world, ms_max)
+    alpha = None if name in TREES else empirical_alpha(acc, sets[0].k)
     step_s = ms_max / 1e3 / args.steps
     peak, peak_src = _peaks()
     achieved = alg_bytes / step_s / 1e9
@@ -464,7 +479,9 @@ def run_ours(args, rank, world, local):
             "gpu_launches": runners[0].kernels_per_call * args.steps,
             "clocks": clk.summary(),
             "tokens_per_s": tokens_per_s,
+            "requests_per_s": requests_per_s,
             "mean_accepted": float(np.mean(acc)),
+            "alpha_empirical": alpha,
         }
         if args.cpu_baseline and world == 1:
             line["cpu_baseline"] = oracle_baseline(name, sets[0], rows)

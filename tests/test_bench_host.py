@@ -65,3 +65,16 @@ def test_translation_units():
     assert "sv_walk.cuh" not in main and "walk.cu" not in main
     assert bench.tu_files("walk.cu") == ["sv_common.cuh", "sv_walk.cuh", "walk.cu"]
     assert bench.tu_digest("walk.cu") != bench.tu_digest("specverify.cu")
+
+
+def test_empirical_alpha():
+    a = bench.empirical_alpha([0, 1, 2, 2, 3, -1], 5)
+    assert a[0] == 4 / 5 and a[1] == 3 / 4 and a[2] == 1 / 3 and a[3] == 0.0 and a[4] is None
+    assert bench.empirical_alpha([], 2) == [None, None]
+    # all drafts kept: every position accepts
+    assert bench.empirical_alpha([5, 5, 5], 5) == [1.0] * 5
+
+
+def test_whole_job_rates():
+    # 64 requests a step, 10 steps, 2 ranks, 5 ms: requests and rows per second
+    assert bench.whole_job_rate(64, 10, 2, 5.0) == 64 * 10 * 2 / 0.005
