@@ -54,6 +54,9 @@ def lib():
         L.orc_verify_tree_u.argtypes = [_P, _P, _I, _I64, _P, _P, _I, _I, _I, _I, _I, _D,
                                         _P, _P, _P, _P, _P, _P, _P, _P]
         L.orc_verify_tree_u.restype = _I
+        L.orc_verify_tree_exact_u.argtypes = [_P, _P, _I, _I64, _P, _P, _I, _I, _I, _I, _D,
+                                              _P, _P, _P, _P, _P, _P, _P, _P]
+        L.orc_verify_tree_exact_u.restype = _I
         L.orc_log_softmax_row.argtypes = [_P, _I, _I, _D, _P]
         L.orc_log_softmax_row.restype = _I
         _lib = L
@@ -197,6 +200,42 @@ def verify_tree(target, draft, node_tokens, parents, max_depth, vocab, stochasti
     ua, us = tree_uniforms(seed, offset, B, N)
     return verify_tree_u(target, draft, node_tokens, parents, max_depth, vocab, stochastic,
                          temperature, ua, us)
+
+
+def verify_tree_exact_u(target, draft, node_tokens, parents, max_depth, vocab, temperature,
+                        u_accept, u_sample):
+    """Distribution-exact tree verification (recursive rejection over
+    siblings) with given uniforms: u_accept [B][N] (entry c tests node c),
+    u_sample [B][N] (entry d draws at node d).  Same outputs as
+    verify_tree_u."""
+    t, dt = _logits(target)
+    d, dd = _logits(draft)
+    assert dd == dt and d.shape == t.shape
+    B, N, stride = t.shape
+    tk = np.ascontiguousarray(node_tokens, dtype=np.int32).reshape(B, N)
+    pa = np.ascontiguousarray(parents, dtype=np.int32).reshape(B, N)
+    ua = np.ascontiguousarray(u_accept, dtype=np.float64).reshape(B, N)
+    us = np.ascontiguousarray(u_sample, dtype=np.float64).reshape(B, N)
+    W = max_depth + 1
+    r = dict(out=np.zeros((B, W), np.int32), acc=np.zeros(B, np.int32),
+             path=np.zeros((B, W), np.int32), acc_margin=np.zeros((B, N)),
+             smp_margin=np.zeros(B), err=np.zeros(B, np.int32))
+    rc = lib().orc_verify_tree_exact_u(_ptr(t), _ptr(d), dt, stride, _ptr(tk), _ptr(pa), B, N,
+                                       max_depth, vocab, float(temperature), _ptr(ua), _ptr(us),
+                                       _ptr(r["out"]), _ptr(r["acc"]), _ptr(r["path"]),
+                                       _ptr(r["acc_margin"]), _ptr(r["smp_margin"]),
+                                       _ptr(r["err"]))
+    if rc != 0:
+        raise ValueError(f"oracle verify_tree_exact rejected its arguments ({rc})")
+    return r
+
+
+def verify_tree_exact(target, draft, node_tokens, parents, max_depth, vocab, temperature, seed,
+                      offset):
+    B, N = np.asarray(target).shape[:2]
+    ua, us = tree_uniforms(seed, offset, B, N)
+    return verify_tree_exact_u(target, draft, node_tokens, parents, max_depth, vocab,
+                               temperature, ua, us)
 
 
 def log_softmax_row(row, temperature):

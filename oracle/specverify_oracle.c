@@ -493,6 +493,137 @@ int orc_verify_tree_u(const void *tl, const void *dl, int dtype, int64_t stride,
     return 0;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Distribution-exact tree verification: recursive rejection over siblings. */
+/* The pages give the tree ([Sonar] "EAGLE") and the single-draft rule      */
+/* ([Leviathan], [Explainer] "Draft and verification loop"); this mode      */
+/* applies that rule to one sibling after another.  Walk from the root; at  */
+/* node u, with p the current target distribution (first p_u) and q_u the   */
+/* draft distribution u's children were drawn from, test u's children in    */
+/* index order against the current p:                                       */
+/*   child c, token t, accepted <=> u_acc[c] * q_u(t) < p(t);               */
+/*   accepted: c becomes the node (p = p_c) and its children are tested;    */
+/*   rejected: p = norm(max(0, p - q_u)) ([Leviathan]'s residual), and the  */
+/*   next sibling is tested against it.                                     */
+/* When u has no child left (or none), the final token is drawn from the    */
+/* current p by the inverse CDF with u_smp[u].  If the children of every    */
+/* node are independent draws from q_u, the emitted tokens follow the       */
+/* target's distribution, each rejection round being one speculative-       */
+/* sampling step against the residual of the last.  Readings: a zero        */
+/* residual mass (reachable only through rounding) leaves p unchanged; the  */
+/* uniforms are those of orc_verify_tree_u (test of node c: u_acc[c]; draw  */
+/* at node d: u_smp[d]).  p is kept as unnormalised weights and their sum,  */
+/* so that on a chain every number equals the linear mode's.                */
+/* Inputs, checks and outputs as orc_verify_tree_u (stochastic);            */
+/* acc_margin[c] holds the margin of every tested child (+inf untested).    */
+/* ------------------------------------------------------------------------ */
+int orc_verify_tree_exact_u(const void *tl, const void *dl, int dtype, int64_t stride,
+                            const int32_t *tokens, const int32_t *parents, int B, int N,
+                            int max_depth, int V, double T, const double *u_acc,
+                            const double *u_smp, int32_t *out, int32_t *acc, int32_t *path,
+                            double *acc_margin, double *smp_margin, int32_t *err)
+{
+    if (B < 0 || N < 1 || V < 1 || max_depth < 1 || !(T > 0.0)) return -1;
+    int *depth = (int *)malloc(sizeof(int) * (size_t)N);
+    int *has_child = (int *)malloc(sizeof(int) * (size_t)N);
+    row_stats *ts = (row_stats *)malloc(sizeof(row_stats) * (size_t)N);
+    row_stats *ds = (row_stats *)malloc(sizeof(row_stats) * (size_t)N);
+    double *cur = (double *)malloc(sizeof(double) * (size_t)V);
+    double *w = (double *)malloc(sizeof(double) * (size_t)V);
+    if (!depth || !has_child || !ts || !ds || !cur || !w) {
+        free(depth); free(has_child); free(ts); free(ds); free(cur); free(w);
+        return -2;
+    }
+    const int W = max_depth + 1;
+    for (int b = 0; b < B; ++b) {
+        const int32_t *tk = tokens + (int64_t)b * N;
+        const int32_t *pa = parents + (int64_t)b * N;
+        int32_t e = 0;
+        smp_margin[b] = INFINITY;
+        for (int i = 0; i < N; ++i) acc_margin[(int64_t)b * N + i] = INFINITY;
+        if (pa[0] != -1) e |= ORC_ERR_TREE;
+        depth[0] = 0;
+        for (int i = 0; i < N; ++i) has_child[i] = 0;
+        for (int i = 1; i < N; ++i) {
+            if (pa[i] < 0 || pa[i] >= i) {
+                e |= ORC_ERR_TREE;
+                depth[i] = 0;
+                continue;
+            }
+            depth[i] = depth[pa[i]] + 1;
+            if (depth[i] > max_depth) e |= ORC_ERR_TREE;
+            has_child[pa[i]] = 1;
+            if (tk[i] < 0 || tk[i] >= V) e |= ORC_ERR_TOKEN;
+        }
+        if (!(e & ORC_ERR_TREE)) {
+            for (int i = 0; i < N; ++i) {
+                int64_t off = ((int64_t)b * N + i) * stride;
+                ts[i] = softmax_stats(tl, dtype, off, V, T);
+                if (ts[i].bad) e |= ORC_ERR_LOGIT;
+                if (has_child[i]) {
+                    ds[i] = softmax_stats(dl, dtype, off, V, T);
+                    if (ds[i].bad) e |= ORC_ERR_LOGIT;
+                }
+            }
+        }
+        err[b] = e;
+        int32_t *ob = out + (int64_t)b * W;
+        int32_t *pb = path ? path + (int64_t)b * W : NULL;
+        for (int j = 0; j < W; ++j) {
+            ob[j] = -1;
+            if (pb) pb[j] = -1;
+        }
+        if (e) {
+            acc[b] = -1;
+            continue;
+        }
+        int u = 0;
+        for (;;) {
+            /* p = target row of u: weights exp((l - m)/T), total S */
+            int64_t toff = ((int64_t)b * N + u) * stride;
+            for (int v = 0; v < V; ++v) cur[v] = exp((logit_at(tl, dtype, toff + v) - ts[u].m) / T);
+            double Zc = ts[u].S;
+            int residual = 0; /* cur holds a residual (not the target row) */
+            int next = -1;
+            for (int c = u + 1; c < N && next < 0; ++c) {
+                if (pa[c] != u) continue;
+                int t = tk[c];
+                double lq = log_prob(dl, dtype, toff, ds[u], t, T);
+                double lp = residual ? log(cur[t] / Zc) : log_prob(tl, dtype, toff, ts[u], t, T);
+                if (accept_test(lp, lq, u_acc[(int64_t)b * N + c], &acc_margin[(int64_t)b * N + c])) {
+                    next = c;
+                    break;
+                }
+                /* [Leviathan] residual of the current p against q_u */
+                double Z = 0.0;
+                for (int v = 0; v < V; ++v) {
+                    double pv = cur[v] / Zc;
+                    double qv = exp((logit_at(dl, dtype, toff + v) - ds[u].m) / T) / ds[u].S;
+                    w[v] = pv > qv ? pv - qv : 0.0;
+                    Z += w[v];
+                }
+                if (Z > 0.0) { /* zero residual mass (rounding only): p unchanged */
+                    for (int v = 0; v < V; ++v) cur[v] = w[v];
+                    Zc = Z;
+                    residual = 1;
+                }
+            }
+            if (next < 0) break;
+            u = next;
+        }
+        int D = depth[u];
+        for (int node = u; node != 0; node = pa[node]) {
+            ob[depth[node] - 1] = tk[node];
+            if (pb) pb[depth[node]] = node;
+        }
+        if (pb) pb[0] = 0;
+        ob[D] = inverse_cdf(cur, V, u_smp[(int64_t)b * N + u], &smp_margin[b]);
+        acc[b] = D;
+    }
+    free(depth); free(has_child); free(ts); free(ds); free(cur); free(w);
+    return 0;
+}
+
 /* Row statistics helper exposed for tests: log-softmax of one row. */
 int orc_log_softmax_row(const void *row, int dtype, int V, double T, double *out_logp)
 {
