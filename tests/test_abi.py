@@ -133,3 +133,21 @@ def test_walk_host_validation(lib):
     assert t(depth=0) == SPEC_EINVAL and t(batch=-2) == SPEC_EINVAL
     assert t(par=0) == SPEC_EINVAL and t(tl=0x1002) == SPEC_EALIGN
     assert t(batch=0) == SPEC_OK and t(batch=0, tl=0, par=0) == SPEC_OK
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    # the product path has no fallback: a missing library is an error, and
+    # the binding never imports the oracle
+    import subprocess
+    import sys
+    code = (
+        "import sys; sys.path.insert(0, %r)\n"
+        "from speculative_decoding_verification_87_b200 import binding\n"
+        "try:\n"
+        "    binding.load_library(%r)\n"
+        "except binding.SpecVerifyError as e:\n"
+        "    print('raised', 'missing' in str(e))\n"
+        "print('oracle' in sys.modules)\n" % (ROOT, str(tmp_path / "absent.so")))
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                         timeout=120).stdout.split()
+    assert out == ["raised", "True", "False"], out
