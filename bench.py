@@ -50,6 +50,7 @@ KERNEL_OF = {
 WALKS = ("greedy-walk", "tree-walk")
 TREES = ("tree", "tree-stochastic", "tree-walk")
 L2_BYTES = 126 * 2 ** 20
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal (context beside the measured peak)
 
 
 CSRC = os.path.join(ROOT, "speculative_decoding_verification_87_b200", "csrc")
@@ -474,7 +475,8 @@ def run_ours(args, rank, world, local):
                          "kernel": KERNEL_OF.get(name, "verification call"),
                          "timed": "CUDA events around each call on its stream (all of the call's "
                                   "kernels, which run back to back)",
-                         "algorithmic_bytes_per_launch": alg_bytes},
+                         "algorithmic_bytes_per_launch": alg_bytes,
+                         "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS},
             "e2e": e2e,
             "gpu_launches": runners[0].kernels_per_call * args.steps,
             "clocks": clk.summary(),
