@@ -3,7 +3,9 @@ over siblings): hand-worked cases, equality with the linear mode on chain
 trees, the root-only draw, input errors, and a chi-square over 1e6 trials
 showing that the emitted tokens follow the target distribution when every
 node's children are independent draws from its draft distribution (with a
-negative control: the independent-test tree mode fails the same test)."""
+negative control: the independent-test tree mode fails the same test), and
+the closed form of a chain of rejections: after r rejections the residual
+is norm(max(0, p - c_r q)), one threshold per node."""
 import numpy as np
 from scipy import stats
 
@@ -178,3 +180,60 @@ def test_emitted_tokens_follow_the_target_distribution(orc):
     # accepted one is biased, and the same test sees it
     pval_ind, _ = _emitted_chi2(np.concatenate(outs_ind), np.concatenate(accs_ind), tabs)
     assert pval_ind < 1e-6, pval_ind
+
+
+# ------------------------------------------------- residual chain closed form
+def _nested(p, q, r):
+    """r literal residual steps: p <- norm(max(0, p - q))."""
+    for _ in range(r):
+        w = np.maximum(p - q, 0.0)
+        p = w / w.sum()
+    return p
+
+
+def _collapsed(p, q, r):
+    """The same as one threshold: norm(max(0, p - c q)) with c_1 = 1 and
+    c_{i+1} = c_i + D_i, D_i = sum(max(0, p - c_i q))."""
+    c = 1.0
+    for _ in range(r - 1):
+        c += np.maximum(p - c * q, 0.0).sum()
+    w = np.maximum(p - c * q, 0.0)
+    return w / w.sum(), c
+
+
+def test_residual_chain_is_one_threshold():
+    rng = np.random.default_rng(21)
+    for _ in range(50):
+        V = int(rng.integers(5, 80))
+        p = softmax64(rng.normal(0, 2, V), 1.0)
+        q = softmax64(rng.normal(0, 2, V), 1.0)
+        for r in (1, 2, 3, 4):
+            a = _nested(p, q, r)
+            if not np.isfinite(a).all():  # the mass ran out (p <= c q everywhere)
+                break
+            b, _ = _collapsed(p, q, r)
+            assert np.allclose(a, b, rtol=1e-10, atol=1e-14)
+
+
+def test_oracle_draw_after_rejections_matches_the_closed_form(orc):
+    # a root whose children all carry a token of zero residual mass are all
+    # rejected whatever u; the final draw then comes from norm(max(0, p - c q))
+    rng = np.random.default_rng(33)
+    V, K = 40, 3
+    P = rng.normal(0, 2, V)
+    Q = P + rng.normal(0, 1.5, V)
+    p, q = softmax64(P.astype(np.float32), 1.0), softmax64(Q.astype(np.float32), 1.0)
+    dead = int(np.argmin(p - q))  # p < q here, so p - c q < 0 for every c >= 1
+    assert p[dead] - q[dead] < 0
+    M = 400
+    tl = np.tile(P.astype(np.float32), (M, K + 1, 1))
+    dl = np.tile(Q.astype(np.float32), (M, K + 1, 1))
+    tok = np.full((M, K + 1), dead, np.int32)
+    par = np.zeros((M, K + 1), np.int32)
+    par[:, 0] = -1
+    us = rng.random((M, K + 1))
+    r = orc.verify_tree_exact_u(tl, dl, tok, par, 1, V, 1.0, np.full((M, K + 1), 0.5), us)
+    assert (r["acc"] == 0).all()
+    w, _ = _collapsed(p, q, K)  # K rejections: K residual steps
+    want = np.searchsorted(np.cumsum(w), us[:, 0], side="right")
+    assert np.array_equal(r["out"][:, 0], want)
