@@ -23,7 +23,7 @@ import numpy as np
 from . import build as _build
 
 ACCEPT, SAMPLE, DRAFT = 0, 1, 2
-ERR_TOKEN, ERR_TREE, ERR_LOGIT = 1, 2, 4
+ERR_TOKEN, ERR_TREE, ERR_LOGIT, ERR_CAPACITY = 1, 2, 4, 16
 
 _lib = None
 
@@ -59,6 +59,8 @@ def lib():
         L.orc_verify_tree_exact_u.restype = _I
         L.orc_log_softmax_row.argtypes = [_P, _I, _I, _D, _P]
         L.orc_log_softmax_row.restype = _I
+        L.orc_plug_tokens.argtypes = [_P, _P, _P, _I, _I, _P, _P, _P, _I]
+        L.orc_plug_tokens.restype = _I
         _lib = L
     return _lib
 
@@ -245,3 +247,23 @@ def log_softmax_row(row, temperature):
     if rc != 0:
         raise ValueError("row has no finite normaliser")
     return out
+
+
+def plug_tokens(in_tokens, out_tokens, accepted_len, seq_tokens=None, seq_len=None,
+                want_next=True):
+    """Device-side token plug of the next step's inputs (see the C source).
+    in_tokens, out_tokens [B][k+1]; accepted_len [B]; seq_tokens [B][cap]
+    and seq_len [B] are copied, updated and returned.  Returns a dict with
+    next [B][k+1] (or None), seq, len and the error bits."""
+    a = np.ascontiguousarray(in_tokens, dtype=np.int32)
+    B, W = a.shape
+    k = W - 1
+    o = np.ascontiguousarray(out_tokens, dtype=np.int32).reshape(B, W)
+    n = np.ascontiguousarray(accepted_len, dtype=np.int32).reshape(B)
+    nxt = np.zeros((B, W), np.int32) if want_next else None
+    seq = None if seq_tokens is None else np.array(seq_tokens, dtype=np.int32, copy=True)
+    ln = None if seq_len is None else np.array(seq_len, dtype=np.int32, copy=True).reshape(B)
+    cap = 0 if seq is None else seq.shape[1]
+    bits = lib().orc_plug_tokens(_ptr(a), _ptr(o), _ptr(n), B, k, _ptr(nxt), _ptr(seq), _ptr(ln),
+                                 cap)
+    return dict(next=nxt, seq=seq, len=ln, err=int(bits))

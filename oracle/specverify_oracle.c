@@ -632,3 +632,58 @@ int orc_log_softmax_row(const void *row, int dtype, int V, double T, double *out
     for (int v = 0; v < V; ++v) out_logp[v] = log_prob(row, dtype, 0, st, v, T);
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* [Sonar] "MTP schedule for one token": after verification a kernel plugs  */
+/* the next target tokens into their positions, so that the accepted count  */
+/* never has to reach the CPU before the next step; "MTP": the draft reads  */
+/* the target's input tokens shifted one step left of its hidden states    */
+/* (the token at position i is the one that follows position i).           */
+/*                                                                          */
+/* Per request b with n = acc[b] and emitted tokens e_0..e_n = out[b][0..n]: */
+/*   next[b][i] = in[b][i + 1] for i < k, i != n (the shifted input; for    */
+/*                i > n these are drafts after the first rejection, a       */
+/*                don't-care the next draft run processes and discards);    */
+/*   next[b][n] = e_n (the drawn token plugged at its position);            */
+/*   next[b][k] = e_n when n < k (no shifted token is left there: a pad);   */
+/*   seq[b][len[b] + j] = e_j for j <= n, then len[b] += n + 1.             */
+/* n = -1 (a request the verification reported as an error): no change to  */
+/* seq, next[b][*] = -1.  n outside [-1, k]: the same, plus the token error  */
+/* bit.  A sequence without room for n + 1 more tokens (or a negative        */
+/* length): seq and len unchanged, next as above, plus ORC_ERR_CAPACITY.    */
+/* next and seq may be NULL (then that part is skipped).  Returns the OR of */
+/* the error bits (0: none).                                                */
+#define ORC_ERR_CAPACITY 16
+int orc_plug_tokens(const int32_t *in, const int32_t *out, const int32_t *acc, int B, int k,
+                    int32_t *next, int32_t *seq, int32_t *len, int capacity)
+{
+    int bits = 0;
+    for (int b = 0; b < B; ++b) {
+        const int32_t *inb = in + (int64_t)b * (k + 1);
+        const int32_t *e = out + (int64_t)b * (k + 1);
+        int32_t *nb = next ? next + (int64_t)b * (k + 1) : NULL;
+        const int n = acc[b];
+        if (n < 0 || n > k) {
+            if (n != -1) bits |= ORC_ERR_TOKEN;
+            if (nb)
+                for (int i = 0; i <= k; ++i) nb[i] = -1;
+            continue;
+        }
+        if (nb) {
+            for (int i = 0; i < k; ++i) nb[i] = inb[i + 1];
+            nb[k] = e[n];
+            nb[n] = e[n];
+        }
+        if (seq) {
+            const int L = len[b];
+            if (L < 0 || (int64_t)L + n + 1 > (int64_t)capacity) {
+                bits |= ORC_ERR_CAPACITY;
+                continue;
+            }
+            int32_t *sb = seq + (int64_t)b * capacity;
+            for (int j = 0; j <= n; ++j) sb[L + j] = e[j];
+            len[b] = L + n + 1;
+        }
+    }
+    return bits;
+}
