@@ -1,4 +1,6 @@
 """Statistical helpers shared by the oracle and GPU distribution tests."""
+import itertools
+
 import numpy as np
 from scipy import stats
 
@@ -38,3 +40,30 @@ def softmax64(logits, temperature):
     z = z - z.max(axis=-1, keepdims=True)
     e = np.exp(z)
     return e / e.sum(axis=-1, keepdims=True)
+
+
+def brute_force_linear(p, q, k):
+    """Exact distribution of (n, emitted tokens) by enumerating all drafts."""
+    V = p.shape[-1]
+    dist = {}
+    for xs in itertools.product(range(V), repeat=k):
+        wx = np.prod([q[j, xs[j]] for j in range(k)])
+        if wx == 0:
+            continue
+        r = [min(1.0, p[j, xs[j]] / q[j, xs[j]]) for j in range(k)]
+        reach = wx
+        for m in range(k + 1):
+            if m < k:
+                pm = reach * (1 - r[m])
+                res = np.maximum(p[m] - q[m], 0)
+                res = res / res.sum() if res.sum() > 0 else p[m]
+            else:
+                pm = reach
+                res = p[k]
+            for y in range(V):
+                if pm * res[y] > 0:
+                    key = (m,) + tuple(xs[:m]) + (y,)
+                    dist[key] = dist.get(key, 0.0) + pm * res[y]
+            if m < k:
+                reach *= r[m]
+    return dist

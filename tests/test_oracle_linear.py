@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 
 from speculative_decoding_verification_87_b200 import workloads as wl
-from stats_util import chisquare_pvalue, softmax64
+from stats_util import brute_force_linear, chisquare_pvalue, softmax64
 
 LN = np.log
 
@@ -226,33 +226,6 @@ def test_chi_square_tiny_config_1e6_trials(orc):
         assert bad == 0 and pv > 1e-3, (b, pv)
 
 
-def _brute_force_linear(p, q, k):
-    """Exact distribution of (n, emitted tokens) by enumerating all drafts."""
-    V = p.shape[-1]
-    dist = {}
-    for xs in itertools.product(range(V), repeat=k):
-        wx = np.prod([q[j, xs[j]] for j in range(k)])
-        if wx == 0:
-            continue
-        r = [min(1.0, p[j, xs[j]] / q[j, xs[j]]) for j in range(k)]
-        reach = wx
-        for m in range(k + 1):
-            if m < k:
-                pm = reach * (1 - r[m])
-                res = np.maximum(p[m] - q[m], 0)
-                res = res / res.sum() if res.sum() > 0 else p[m]
-            else:
-                pm = reach
-                res = p[k]
-            for y in range(V):
-                if pm * res[y] > 0:
-                    key = (m,) + tuple(xs[:m]) + (y,)
-                    dist[key] = dist.get(key, 0.0) + pm * res[y]
-            if m < k:
-                reach *= r[m]
-    return dist
-
-
 def test_brute_force_rule_keeps_target_joint():
     """The accept/residual rule itself (not the oracle) reproduces the
     target's autoregressive joint: an exact check of the guarantee."""
@@ -260,7 +233,7 @@ def test_brute_force_rule_keeps_target_joint():
     V, k = 8, 2
     p = softmax64(rng.normal(0, 1.5, (k + 1, V)), 1.0)
     q = softmax64(np.log(p[:k]) + rng.normal(0, 0.7, (k, V)), 1.0)
-    dist = _brute_force_linear(p, q, k)
+    dist = brute_force_linear(p, q, k)
     assert abs(sum(dist.values()) - 1) < 1e-12
     for j in range(k + 1):
         for z in itertools.product(range(V), repeat=j):
@@ -277,7 +250,7 @@ def test_brute_force_v8_k2_matches_oracle(orc):
     base = wl.tiny_linear(seed=21, batch=1, k=k, vocab=V)
     p = softmax64(wl.as_f32(base.target, V), T)[0]
     q = softmax64(wl.as_f32(base.draft, V), T)[0]
-    dist = _brute_force_linear(p, q, k)
+    dist = brute_force_linear(p, q, k)
     keys = sorted(dist)
     index = {key: i for i, key in enumerate(keys)}
     outs, accs = _trials(orc, base, 400_000, 4)
