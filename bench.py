@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--config batched|single|greedy|tree|tree-stochastic|
-                              greedy-walk|tree-walk]
+                              tree-exact|greedy-walk|tree-walk] [--l2 cold|warm]
 
 A step is one verification call over one batch of synthetic inputs: for the
 default workload, 64 requests x 8 drafts over a 128256-entry bf16
@@ -44,11 +44,14 @@ KERNEL_OF = {
     "greedy": "k_greedy_cluster (one launch per call)",
     "tree": "k_pass1 + k_decide (programmatic dependents)",
     "tree-stochastic": "k_pass1 + k_decide + k_pass2 + k_finalize (programmatic dependents)",
+    "tree-exact": "k_pass1 + k_tree_exact (programmatic dependent)",
     "greedy-walk": "k_greedy_walk (one launch per call)",
     "tree-walk": "k_greedy_walk (one launch per call)",
 }
 WALKS = ("greedy-walk", "tree-walk")
-TREES = ("tree", "tree-stochastic", "tree-walk")
+TREES = ("tree", "tree-stochastic", "tree-exact", "tree-walk")
+STOCH_TREES = {"tree-stochastic": 1, "tree-exact": 2}
+READS_DRAFTS = ("batched", "single", "tree-stochastic", "tree-exact")
 L2_BYTES = 126 * 2 ** 20
 NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal (context beside the measured peak)
 
@@ -171,11 +174,12 @@ def workload_facts(name, w):
     else:
         B, N, V = w.batch, w.num_nodes, w.vocab
         rows = B * N
-        stoch = name == "tree-stochastic"
+        stoch = name in STOCH_TREES
         nonleaf = sum(int(len(set(w.parents[b, 1:].tolist()))) for b in range(B))
         logits = (B * N + (nonleaf if stoch else 0)) * V * esz
         io = 2 * B * N * 4 + 2 * B * (w.max_depth + 1) * 4 + B * 4
-        cfg = dict(workload=f"tree {'stochastic' if stoch else 'greedy'} verify B={B} N={N} "
+        mode = {"tree-exact": "exact stochastic", "tree-stochastic": "stochastic"}.get(name, "greedy")
+        cfg = dict(workload=f"tree {mode} verify B={B} N={N} "
                             f"depth={w.max_depth} V={V} {w.dtype}", batch=B, nodes=N, vocab=V)
     return rows, logits + io, cfg
 
@@ -184,7 +188,7 @@ def workload_facts(name, w):
 class ClockSampler:
     """Samples SM clock and throttle reasons through NVML while running."""
 
-    def __init__(self, index, period=0.01):
+    def __init__(self, index, period=0.001):
         self.index, self.period = index, period
         self.samples = []
         self._stop = threading.Event()
@@ -340,7 +344,7 @@ class Runner:
             self.out = torch.empty((w.batch, W), dtype=torch.int32, device=device)
             # pass 1 + decide, then pass 2 + finalize for the stochastic draw;
             # the walk is one kernel
-            self.kernels_per_call = {"tree-stochastic": 4, "tree": 2}.get(name, 1)
+            self.kernels_per_call = {"tree-stochastic": 4, "tree": 2, "tree-exact": 2}.get(name, 1)
         else:
             self.tokens = dev(w.tokens.astype(np.int32))
             self.out = torch.empty((w.batch, w.k + 1), dtype=torch.int32, device=device)
@@ -355,7 +359,7 @@ class Runner:
         import copy
         c = copy.copy(self)
         c.target = self.target.clone()
-        if self.name in ("batched", "single", "tree-stochastic"):  # the modes that read drafts
+        if self.name in READS_DRAFTS:
             c.draft = self.draft.clone()
         c.out = torch_empty_like(self.out)
         c.acc = torch_empty_like(self.acc)
@@ -380,7 +384,7 @@ class Runner:
                                            out_tokens=self.out, accepted_len=self.acc)
         else:
             b.spec_verify_tree(target, draft, tokens, self.parents, w.max_depth, w.vocab,
-                               self.name == "tree-stochastic", w.temperature, 1234, offset,
+                               STOCH_TREES.get(self.name, 0), w.temperature, 1234, offset,
                                out_tokens=self.out, accepted_len=self.acc)
 
 
@@ -409,6 +413,8 @@ def run_ours(args, rank, world, local):
     n_cycle += n_cycle % 2
     while len(runners) < n_cycle:
         runners.append(runners[len(runners) % 2].clone())
+    if args.l2 == "warm":
+        runners = runners[:1]
     stream = torch.cuda.current_stream(device)
 
     # warm-up
@@ -463,9 +469,11 @@ def run_ours(args, rank, world, local):
             "dtype": sets[0].dtype,
             "data": "synthetic",
             "config": dict(cfg, parallelism=f"dp{world} (independent request shards)",
-                           l2=f"inputs larger than L2: calls cycle over {len(runners)} resident "
-                              f"input sets (2 seeds, copies at distinct addresses), "
-                              f"{alg_bytes / 1e6:.1f} MB read per call",
+                           l2=(f"inputs larger than L2: calls cycle over {len(runners)} resident "
+                               f"input sets (2 seeds, copies at distinct addresses), "
+                               f"{alg_bytes / 1e6:.1f} MB read per call") if args.l2 == "cold" else
+                              (f"L2 warm: every call reads the same input set "
+                               f"({alg_bytes / 1e6:.1f} MB per call)"),
                            requests_per_rank=sets[0].batch),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
@@ -479,7 +487,8 @@ def run_ours(args, rank, world, local):
                          "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS},
             "e2e": e2e,
             "gpu_launches": runners[0].kernels_per_call * args.steps,
-            "clocks": clk.summary(),
+            "clocks": dict(clk.summary(), kcycles_per_step=(
+                ms_max / args.steps * clk.summary()["sm_mhz"] if clk.summary()["sm_mhz"] else None)),
             "tokens_per_s": tokens_per_s,
             "requests_per_s": requests_per_s,
             "mean_accepted": float(np.mean(acc)),
@@ -503,7 +512,7 @@ def run_e2e(args, runner, w, device, world):
     tok_d = torch.empty(tok_h.shape, dtype=tok_h.dtype, device=device)
     out_h = torch.empty(runner.out.shape, dtype=torch.int32).pin_memory()
     acc_h = torch.empty(runner.acc.shape, dtype=torch.int32).pin_memory()
-    needs_draft = runner.name in ("batched", "single", "tree-stochastic")
+    needs_draft = runner.name in READS_DRAFTS
     stream = torch.cuda.current_stream(device)
 
     def step(i):
@@ -532,8 +541,13 @@ def run_e2e(args, runner, w, device, world):
     if needs_draft:
         h2d += drf_h.numel() * drf_h.element_size()
     d2h = (out_h.numel() + acc_h.numel()) * 4
+    step_ms = ms / steps
     return {"value": rows * steps * world / (ms / 1e3), "unit": "rows/s",
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps}
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "ms_per_step": step_ms,
+            "bound": (f"host-to-device copy: {h2d / 1e6:.1f} MB of logits per step from pinned "
+                      f"memory ({h2d / (step_ms * 1e-3) / 1e9:.1f} GB/s including the call), "
+                      f"not the kernel")}
 
 
 # ------------------------------------------------------------ oracle timing
@@ -559,6 +573,10 @@ def oracle_call(name, s, offset):
         return s.target.shape[0] * s.target.shape[1]
     if name in ("greedy", "greedy-walk"):
         oracle.verify_greedy(s.target, s.tokens, s.vocab)
+        return s.target.shape[0] * s.target.shape[1]
+    if name == "tree-exact":
+        oracle.verify_tree_exact(s.target, s.draft, s.node_tokens, s.parents, s.max_depth, s.vocab,
+                                 s.temperature, 1234, offset)
         return s.target.shape[0] * s.target.shape[1]
     oracle.verify_tree(s.target, s.draft, s.node_tokens, s.parents, s.max_depth, s.vocab,
                        name == "tree-stochastic", s.temperature, 1234, offset)
@@ -645,9 +663,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="batched",
-                    choices=["batched", "single", "greedy", "tree", "tree-stochastic",
+                    choices=["batched", "single", "greedy", "tree", "tree-stochastic", "tree-exact",
                              "greedy-walk", "tree-walk"])
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--l2", choices=["cold", "warm"], default="cold",
+                    help="cold: calls cycle over input copies that together exceed L2 (every call "
+                         "reads HBM); warm: every call reads the same inputs (a small workload "
+                         "then reads L2)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -19,12 +19,14 @@ LIB_PATH = os.path.join(_HERE, "libspecverify.so")
 
 SPEC_F32, SPEC_BF16 = 0, 1
 SPEC_OK = 0
-STATUS_TOKEN, STATUS_TREE, STATUS_LOGIT, STATUS_TIMEOUT = 1, 2, 4, 8
+STATUS_TOKEN, STATUS_TREE, STATUS_LOGIT, STATUS_TIMEOUT, STATUS_CAPACITY = 1, 2, 4, 8, 16
 MAX_K, MAX_NODES = 32, 1024
 SYMBOLS = ("spec_verify_workspace_size", "spec_verify_strerror", "spec_verify_linear",
            "spec_verify_greedy", "spec_verify_tree", "spec_verify_debug_uniforms",
            "spec_verify_linear_noalloc", "spec_verify_debug_exp2", "spec_verify_greedy_walk",
-           "spec_verify_tree_greedy_walk")
+           "spec_verify_tree_greedy_walk", "spec_verify_debug_wait_expiry", "spec_plug_tokens",
+           "spec_shard_row_stats", "spec_shard_decide", "spec_shard_decide_greedy",
+           "spec_shard_draw_sums", "spec_shard_draw_pick", "spec_shard_emit")
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 _lib = None
@@ -75,6 +77,26 @@ def load_library(path: str = LIB_PATH):
         L.spec_verify_tree_greedy_walk.restype = _I
         L.spec_verify_debug_exp2.argtypes = [_P, _P, _I, _I, _P]
         L.spec_verify_debug_exp2.restype = _I
+        L.spec_verify_debug_wait_expiry.argtypes = [_P, _P, _I, _I64, _P, _I, _I, _I, _F, _U32,
+                                                    _P, _P, _P, _P, _SZ, _P]
+        L.spec_verify_debug_wait_expiry.restype = _I
+        L.spec_plug_tokens.argtypes = [_P, _P, _P, _I, _I, _P, _P, _P, _I, _P, _P]
+        L.spec_plug_tokens.restype = _I
+        L.spec_shard_row_stats.argtypes = [_P, _P, _I, _I64, _P, _I, _I, _I, _I, _F, _P, _P, _P, _P,
+                                           _P]
+        L.spec_shard_row_stats.restype = _I
+        L.spec_shard_decide.argtypes = [_P, _P, _P, _P, _I, _P, _I, _I, _I, _F, _U64, _U32, _P, _P,
+                                        _P, _P, _P]
+        L.spec_shard_decide.restype = _I
+        L.spec_shard_decide_greedy.argtypes = [_P, _P, _I, _P, _I, _I, _I, _P, _P, _P, _P]
+        L.spec_shard_decide_greedy.restype = _I
+        L.spec_shard_draw_sums.argtypes = [_P, _P, _I, _I64, _I, _I, _I, _I, _F, _P, _P, _I, _P, _P]
+        L.spec_shard_draw_sums.restype = _I
+        L.spec_shard_draw_pick.argtypes = [_P, _P, _I, _I64, _I, _I, _I, _I, _F, _P, _P, _P, _I, _I,
+                                           _P, _P]
+        L.spec_shard_draw_pick.restype = _I
+        L.spec_shard_emit.argtypes = [_P, _P, _I, _I, _P, _P]
+        L.spec_shard_emit.restype = _I
         _lib = L
         return L
 
@@ -249,8 +271,13 @@ def spec_verify_tree(target_logits, draft_logits, node_tokens, parents, max_dept
                      accepted_len=None, out_path_nodes=None, status=None, workspace_buf=None,
                      stream=None):
     """target_logits [B][N][stride]; draft_logits [B][N][stride] or None (greedy);
-    node_tokens, parents [B][N] int32.  Returns (out_tokens [B][D+1],
+    node_tokens, parents [B][N] int32.  stochastic: 0 (or False) greedy, 1 (or
+    True) an independent test per node, 2 distribution-exact (siblings tested
+    in turn against the residual).  Returns (out_tokens [B][D+1],
     accepted_len [B], out_path_nodes [B][D+1] or None)."""
+    stochastic = int(stochastic)
+    if stochastic not in (0, 1, 2):
+        raise ValueError("stochastic must be 0, 1 or 2")
     _need_cuda("target_logits", target_logits)
     B, N, stride = target_logits.shape
     if stochastic:
@@ -275,7 +302,7 @@ def spec_verify_tree(target_logits, draft_logits, node_tokens, parents, max_dept
     rc = load_library().spec_verify_tree(
         _ptr(target_logits), _ptr(draft_logits if stochastic else None),
         _dtype_code(target_logits), stride, _ptr(node_tokens), _ptr(parents), B, N, max_depth,
-        vocab, int(bool(stochastic)), float(temperature), int(seed), int(offset), _ptr(out_tokens),
+        vocab, int(stochastic), float(temperature), int(seed), int(offset), _ptr(out_tokens),
         _ptr(accepted_len), _ptr(out_path_nodes), _ptr(status), _ptr(workspace_buf), ws_bytes,
         _stream(stream))
     _check(rc, "spec_verify_tree")
@@ -304,6 +331,34 @@ def spec_verify_debug_exp2(z, kind=0, stream=None):
                                                _stream(stream))
     _check(rc, "spec_verify_debug_exp2")
     return out
+
+
+def spec_verify_debug_wait_expiry(target_logits, draft_logits, draft_tokens, vocab, temperature,
+                                  poll_limit, status, out_tokens=None, accepted_len=None,
+                                  workspace_buf=None, stream=None):
+    """spec_verify_linear with its waits made to expire after poll_limit polls
+    (diagnostic: pass 1 stores nothing, so every decide step gives up and
+    reports SPEC_STATUS_TIMEOUT into status; the outputs stay -1)."""
+    _need_cuda("target_logits", target_logits)
+    B, R, stride = target_logits.shape
+    k = R - 1
+    _need_cuda("draft_logits", draft_logits, target_logits.dtype, (B, k, stride))
+    _need_cuda("draft_tokens", draft_tokens, torch.int32, (B, k))
+    _need_cuda("status", status, torch.int32)
+    dev = target_logits.device
+    if out_tokens is None:
+        out_tokens = torch.empty((B, k + 1), dtype=torch.int32, device=dev)
+    if accepted_len is None:
+        accepted_len = torch.empty((B,), dtype=torch.int32, device=dev)
+    if workspace_buf is None:
+        workspace_buf = workspace(B, 2 * k + 1, vocab, dev) if B > 0 else None
+    ws_bytes = 0 if workspace_buf is None else workspace_buf.numel()
+    rc = load_library().spec_verify_debug_wait_expiry(
+        _ptr(target_logits), _ptr(draft_logits), _dtype_code(target_logits), stride,
+        _ptr(draft_tokens), B, k, vocab, float(temperature), int(poll_limit), _ptr(out_tokens),
+        _ptr(accepted_len), _ptr(status), _ptr(workspace_buf), ws_bytes, _stream(stream))
+    _check(rc, "spec_verify_debug_wait_expiry")
+    return out_tokens, accepted_len
 
 
 def spec_verify_linear_noalloc(target_logits, draft_logits, draft_tokens, vocab, temperature,
@@ -336,3 +391,166 @@ def spec_verify_linear_noalloc(target_logits, draft_logits, draft_tokens, vocab,
         _stream(stream))
     _check(rc, "spec_verify_linear_noalloc")
     return out_tokens, accepted_len
+
+
+def spec_plug_tokens(in_tokens, out_tokens, accepted_len, next_tokens=None, seq_tokens=None,
+                     seq_len=None, status=None, stream=None):
+    """Write the next step's input tokens from a verification's outputs on
+    the device (no host synchronisation).  in_tokens, out_tokens [B][k+1],
+    accepted_len [B] int32; next_tokens [B][k+1] (output, allocated when
+    None and want); seq_tokens [B][cap] and seq_len [B] updated in place.
+    Returns next_tokens."""
+    _need_cuda("out_tokens", out_tokens, torch.int32)
+    B, W = out_tokens.shape
+    k = W - 1
+    _need_cuda("in_tokens", in_tokens, torch.int32, (B, W))
+    _need_cuda("accepted_len", accepted_len, torch.int32, (B,))
+    if next_tokens is None:
+        next_tokens = torch.empty((B, W), dtype=torch.int32, device=out_tokens.device)
+    _need_cuda("next_tokens", next_tokens, torch.int32, (B, W))
+    cap = 0
+    if seq_tokens is not None or seq_len is not None:
+        _need_cuda("seq_tokens", seq_tokens, torch.int32)
+        if seq_tokens.dim() != 2 or seq_tokens.shape[0] != B:
+            raise ValueError("seq_tokens must be [B][capacity]")
+        cap = seq_tokens.shape[1]
+        _need_cuda("seq_len", seq_len, torch.int32, (B,))
+    if status is not None:
+        _need_cuda("status", status, torch.int32)
+    rc = load_library().spec_plug_tokens(_ptr(in_tokens), _ptr(out_tokens), _ptr(accepted_len), B,
+                                         k, _ptr(next_tokens), _ptr(seq_tokens), _ptr(seq_len), cap,
+                                         _ptr(status), _stream(stream))
+    _check(rc, "spec_plug_tokens")
+    return next_tokens
+
+
+# ------------------------------------------------------------ vocabulary-sharded steps
+SHARD_DRAW_WORDS = 6
+
+
+def spec_shard_row_stats(target_logits, draft_logits, draft_tokens, vocab_lo, vocab_hi,
+                         temperature=1.0, stream=None):
+    """Per-row statistics of this rank's columns [vocab_lo, vocab_hi).
+    Stochastic (draft_logits given): dict(max [B][2k+1] f32, sum [B][2k+1]
+    f64, probe [B][k][2] f32); greedy (draft_logits None): dict(max
+    [B][k+1] f32, arg [B][k+1] int32)."""
+    _need_cuda("target_logits", target_logits)
+    B, R1, stride = target_logits.shape
+    k = R1 - 1
+    _need_cuda("draft_tokens", draft_tokens, torch.int32, (B, k))
+    dev = target_logits.device
+    stoch = draft_logits is not None
+    if stoch:
+        _need_cuda("draft_logits", draft_logits, target_logits.dtype, (B, k, stride))
+    R = 2 * k + 1 if stoch else k + 1
+    mx = torch.empty((B, R), dtype=torch.float32, device=dev)
+    sm = torch.empty((B, R), dtype=torch.float64, device=dev) if stoch else None
+    arg = None if stoch else torch.empty((B, R), dtype=torch.int32, device=dev)
+    probe = torch.empty((B, k, 2), dtype=torch.float32, device=dev) if stoch else None
+    rc = load_library().spec_shard_row_stats(
+        _ptr(target_logits), _ptr(draft_logits), _dtype_code(target_logits), stride,
+        _ptr(draft_tokens), B, k, int(vocab_lo), int(vocab_hi), float(temperature), _ptr(mx),
+        _ptr(sm), _ptr(arg), _ptr(probe), _stream(stream))
+    _check(rc, "spec_shard_row_stats")
+    return dict(max=mx, sum=sm, arg=arg, probe=probe)
+
+
+def spec_shard_decide(max_all, sum_all, probe_all, bounds, draft_tokens, vocab, temperature,
+                      seed=0, offset=0, status=None, stream=None):
+    """Merge the ranks' statistics (rank order) and run the accept tests.
+    Returns (out_tokens [B][k+1] with the drawn slot still -1,
+    accepted_len [B], draw [B][6] f64)."""
+    _need_cuda("max_all", max_all, torch.float32)
+    W, B, R = max_all.shape
+    k = (R - 1) // 2
+    _need_cuda("sum_all", sum_all, torch.float64, (W, B, R))
+    _need_cuda("probe_all", probe_all, torch.float32, (W, B, k, 2))
+    _need_cuda("bounds", bounds, torch.int32, (W + 1,))
+    _need_cuda("draft_tokens", draft_tokens, torch.int32, (B, k))
+    if status is not None:
+        _need_cuda("status", status, torch.int32)
+    dev = max_all.device
+    out = torch.empty((B, k + 1), dtype=torch.int32, device=dev)
+    acc = torch.empty((B,), dtype=torch.int32, device=dev)
+    draw = torch.empty((B, SHARD_DRAW_WORDS), dtype=torch.float64, device=dev)
+    rc = load_library().spec_shard_decide(
+        _ptr(max_all), _ptr(sum_all), _ptr(probe_all), _ptr(bounds), W, _ptr(draft_tokens), B, k,
+        int(vocab), float(temperature), int(seed), int(offset), _ptr(out), _ptr(acc), _ptr(draw),
+        _ptr(status), _stream(stream))
+    _check(rc, "spec_shard_decide")
+    return out, acc, draw
+
+
+def spec_shard_decide_greedy(max_all, arg_all, draft_tokens, vocab, status=None, stream=None):
+    """Greedy verification from the ranks' (max, lowest argmax) per target row."""
+    _need_cuda("max_all", max_all, torch.float32)
+    W, B, R = max_all.shape
+    k = R - 1
+    _need_cuda("arg_all", arg_all, torch.int32, (W, B, R))
+    _need_cuda("draft_tokens", draft_tokens, torch.int32, (B, k))
+    if status is not None:
+        _need_cuda("status", status, torch.int32)
+    dev = max_all.device
+    out = torch.empty((B, k + 1), dtype=torch.int32, device=dev)
+    acc = torch.empty((B,), dtype=torch.int32, device=dev)
+    rc = load_library().spec_shard_decide_greedy(_ptr(max_all), _ptr(arg_all), W, _ptr(draft_tokens),
+                                                 B, k, int(vocab), _ptr(out), _ptr(acc),
+                                                 _ptr(status), _stream(stream))
+    _check(rc, "spec_shard_decide_greedy")
+    return out, acc
+
+
+def spec_shard_draw_sums(target_logits, draft_logits, vocab_lo, vocab_hi, temperature, draw,
+                         norm_parts=None, stream=None):
+    """fp64 sums over this rank's columns of each request's draw rows:
+    without norm_parts (sum e, sum f); with the ranks' gathered first sums
+    [W][B][2] (the draw mass, sum e).  Returns [B][2] f64."""
+    _need_cuda("target_logits", target_logits)
+    B, R1, stride = target_logits.shape
+    k = R1 - 1
+    _need_cuda("draft_logits", draft_logits, target_logits.dtype, (B, k, stride))
+    _need_cuda("draw", draw, torch.float64, (B, SHARD_DRAW_WORDS))
+    W = 1
+    if norm_parts is not None:
+        _need_cuda("norm_parts", norm_parts, torch.float64)
+        W = norm_parts.shape[0]
+    sums = torch.empty((B, 2), dtype=torch.float64, device=target_logits.device)
+    rc = load_library().spec_shard_draw_sums(
+        _ptr(target_logits), _ptr(draft_logits), _dtype_code(target_logits), stride, B, k,
+        int(vocab_lo), int(vocab_hi), float(temperature), _ptr(draw), _ptr(norm_parts), W,
+        _ptr(sums), _stream(stream))
+    _check(rc, "spec_shard_draw_sums")
+    return sums
+
+
+def spec_shard_draw_pick(target_logits, draft_logits, vocab_lo, vocab_hi, temperature, draw,
+                         norm_parts, mass_parts, shard_index, stream=None):
+    """The token of each request if this rank owns the part of the running
+    mass that holds u * Z (drawn inside its columns), else -1.  [B] int32."""
+    _need_cuda("target_logits", target_logits)
+    B, R1, stride = target_logits.shape
+    k = R1 - 1
+    _need_cuda("draft_logits", draft_logits, target_logits.dtype, (B, k, stride))
+    _need_cuda("draw", draw, torch.float64, (B, SHARD_DRAW_WORDS))
+    _need_cuda("norm_parts", norm_parts, torch.float64)
+    W = norm_parts.shape[0]
+    _need_cuda("mass_parts", mass_parts, torch.float64, (W, B, 2))
+    token = torch.empty((B,), dtype=torch.int32, device=target_logits.device)
+    rc = load_library().spec_shard_draw_pick(
+        _ptr(target_logits), _ptr(draft_logits), _dtype_code(target_logits), stride, B, k,
+        int(vocab_lo), int(vocab_hi), float(temperature), _ptr(draw), _ptr(norm_parts),
+        _ptr(mass_parts), W, int(shard_index), _ptr(token), _stream(stream))
+    _check(rc, "spec_shard_draw_pick")
+    return token
+
+
+def spec_shard_emit(token, draw, out_tokens, stream=None):
+    """out_tokens[b][n] = token[b] for every request that draws one."""
+    _need_cuda("out_tokens", out_tokens, torch.int32)
+    B, W1 = out_tokens.shape
+    _need_cuda("token", token, torch.int32, (B,))
+    _need_cuda("draw", draw, torch.float64, (B, SHARD_DRAW_WORDS))
+    rc = load_library().spec_shard_emit(_ptr(token), _ptr(draw), B, W1 - 1, _ptr(out_tokens),
+                                        _stream(stream))
+    _check(rc, "spec_shard_emit")
+    return out_tokens

@@ -11,7 +11,10 @@
 //
 // Set-up: the first call on a device (with that device current) looks up
 // the array's device address with cudaGetSymbolAddress; later calls reuse
-// it.  Make that first call before any stream capture begins.
+// it for the life of the process.  Make that first call before any stream
+// capture begins.  The cached address does not survive cudaDeviceReset (the
+// module is loaded again into the new context): a device must not be reset
+// while this library may still be called on it.
 // Sharing: all calls on a device use the same array.  Each call clears the
 // counters it needs before use, so stale contents from an earlier call do
 // no harm, but calls that overlap on the GPU (other streams, other host
@@ -62,7 +65,17 @@ extern "C" int spec_verify_linear_noalloc(const void *target_logits, const void 
     void *scratch = nullptr;
     if (batch > 0 && k >= 1) {
         const size_t need = spec_verify_workspace_size(batch, 2 * k + 1, vocab);
-        if (need > kScratchBytes) return SPEC_EUNSUPPORTED;  // beyond the static scratch
+        if (need > kScratchBytes) {
+            // beyond the static scratch; but an invalid argument keeps the
+            // code spec_verify_linear gives it: without a workspace it runs
+            // every other check, enqueues nothing and, if they pass, reports
+            // the workspace
+            const int rc = spec_verify_linear(target_logits, draft_logits, dtype, row_stride,
+                                              draft_tokens, batch, k, vocab, temperature, seed,
+                                              offset, out_tokens, accepted_len, dbg_logp, dbg_logq,
+                                              status, nullptr, 0, stream);
+            return rc == SPEC_EWORKSPACE ? SPEC_EUNSUPPORTED : rc;
+        }
         if (need > 0) {
             const int rc = scratch_address(&scratch);
             if (rc != SPEC_OK) return rc;

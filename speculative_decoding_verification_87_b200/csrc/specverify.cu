@@ -1,7 +1,7 @@
 // specverify.cu -- C ABI of libspecverify.so (sm_100a) and its launches.
 //
-// spec_verify_linear: one memset of the call's counters and pass-1
-// partials, then the persistent kernel k_fused (sv_fused.cuh).
+// spec_verify_linear: one cooperative launch of the persistent kernel
+// k_fused (sv_fused.cuh), which clears its own counters.
 // spec_verify_tree: the pass-1 kernel, the decide kernel and, where a token
 // is drawn, the pass-2 and finalize kernels (sv_verify.cuh), each a
 // programmatic dependent of the one before.
@@ -23,6 +23,7 @@
 #include "sv_fused.cuh"
 #include "sv_exp64.cuh"
 #include "sv_greedy.cuh"
+#include "sv_exact.cuh"
 #include "sv_philox.cuh"
 
 namespace sv {
@@ -39,8 +40,8 @@ __global__ void k_debug_uniforms(uint64_t seed, uint32_t offset, uint32_t purpos
 
 __global__ void k_debug_exp2(const double *z, double *out, int n, int kind, Params p)
 {
-    __shared__ double tab[64];
-    if (threadIdx.x < 64) tab[threadIdx.x] = p.exp2tab[threadIdx.x];
+    __shared__ double tab[kExp2Tab];
+    for (int j = threadIdx.x; j < kExp2Tab; j += blockDim.x) tab[j] = p.exp2tab[j];
     __syncthreads();
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n) return;
@@ -60,9 +61,9 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Workspace layout.  Every region a call reads is written earlier in the
-// same call; the one-kernel path first sets its counters and the pass-1
-// partials (which follow them) to all ones.  Region sizes use the shorter
-// pass-1 item, so both dtypes fit.
+// same call; the one-kernel path first clears its counters and sets the
+// pass-1 partials to all ones.  Region sizes use the shorter pass-1 item,
+// so both dtypes fit.
 struct Layout {
     size_t counters, rowpart, req, p2part, p2amb, ambbits, p2w, p2lane, total;
     bool ok;
@@ -77,8 +78,8 @@ Layout layout(int B, int R, int V)
     const int64_t s2 = ceil_div(V, kSeg2);
     const int64_t w32 = s2 * (kSeg2 / 32);  // whole segments (16-byte aligned rows of the bitmap)
     size_t off = 0;
-    L.counters = off;  // p2cnt[B], decided[B], p2claim, a_claim; rowpart follows directly
-    off = align_up(off + sizeof(unsigned) * (2 * static_cast<size_t>(B) + 2));
+    L.counters = off;  // p2cnt[B], decided[B], rowdone[B][R], p2claim, a_claim, p2ticket
+    off = align_up(off + sizeof(unsigned) * (static_cast<size_t>(B) * (R + 2) + 3));
     L.rowpart = off;
     off = align_up(off + sizeof(float2) * static_cast<size_t>(B) * R * smax);
     L.req = off;
@@ -125,8 +126,11 @@ void fill_workspace(Params &p, void *ws, const Layout &L)
     auto *cnt = reinterpret_cast<unsigned *>(w + L.counters);
     p.p2cnt = cnt;
     p.decided = cnt + p.B;
-    p.p2claim = p.decided + p.B;
+    p.rowdone = p.decided + p.B;
+    p.p2claim = p.rowdone + static_cast<int64_t>(p.B) * p.R;
     p.a_claim = p.p2claim + 1;
+    p.p2ticket = p.a_claim + 1;
+    p.ncounters = static_cast<unsigned>(static_cast<int64_t>(p.B) * (p.R + 2) + 3);
     p.rowpart = reinterpret_cast<float2 *>(w + L.rowpart);
     p.req = reinterpret_cast<ReqInfo *>(w + L.req);
     p.p2part = reinterpret_cast<double4 *>(w + L.p2part);
@@ -136,10 +140,10 @@ void fill_workspace(Params &p, void *ws, const Layout &L)
     p.p2lane = reinterpret_cast<double2 *>(w + L.p2lane);
 }
 
-// 2^(j/64), j = 0..63, from the host math library.
+// 2^(j/256), j = 0..255, from the host math library.
 void fill_exp2_table(Params &p)
 {
-    for (int j = 0; j < 64; ++j) p.exp2tab[j] = std::exp2(static_cast<double>(j) / 64.0);
+    for (int j = 0; j < kExp2Tab; ++j) p.exp2tab[j] = std::exp2(static_cast<double>(j) / kExp2Tab);
 }
 
 
@@ -148,10 +152,17 @@ std::mutex g_mu;
 int g_pass1_blocks[64][2][3];
 int g_pass2_blocks[64][2][3];
 bool g_final_attr[64][2][3];
+bool g_decide_attr[64][2][3];
 int g_sm_count[64];
 
 // Decide dynamic shared memory: the merged statistics of a request's rows.
-size_t decide_smem(int R) { return (sizeof(double) + sizeof(float) + sizeof(int)) * static_cast<size_t>(R); }
+size_t decide_smem(int R, int S)
+{
+    size_t n = (sizeof(double) + sizeof(float) + sizeof(int)) * static_cast<size_t>(R);
+    n = (n + 15) / 16 * 16;
+    if (static_cast<int64_t>(R) * S <= kDecideStageMax) n += sizeof(float2) * static_cast<size_t>(R) * S;
+    return n;
+}
 
 // Finalize dynamic shared memory: the segment weights of each warp, for
 // vocabularies up to kMaxS2Shared segments (else the workspace holds them).
@@ -224,6 +235,15 @@ int launch_verify(Params &p, const Layout &L, void *ws, int dtype_index, cudaStr
     {
         std::lock_guard<std::mutex> lock(g_mu);
         per_sm1 = blocks_per_sm(g_pass1_blocks[dev][dtype_index][MODE], k_pass1<Tag, MODE, kMin1>, kRingBytes);
+        bool &dattr = g_decide_attr[dev][dtype_index][MODE];
+        if (!dattr) {
+            // the largest decide footprint: 2 * kMaxNodes rows' statistics plus staged partials
+            if (cudaFuncSetAttribute(k_decide<Tag, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(decide_smem(2 * kMaxNodes, 0) +
+                                                      sizeof(float2) * kDecideStageMax)) != cudaSuccess)
+                return SPEC_ECUDA;
+            dattr = true;
+        }
         if (p.nP > 0) {
             per_sm2 = blocks_per_sm(g_pass2_blocks[dev][dtype_index][MODE], k_pass2<Tag, MODE>,
                                     StageShape<Tag>::kBytes);
@@ -243,7 +263,7 @@ int launch_verify(Params &p, const Layout &L, void *ws, int dtype_index, cudaStr
     k_pass1<Tag, MODE, kMin1><<<static_cast<unsigned>(blocks1), kThreads, kRingBytes, st>>>(p);
     if (cudaGetLastError() != cudaSuccess) return SPEC_ECUDA;
     const int64_t blocksd = std::max<int64_t>(1, std::min<int64_t>(static_cast<int64_t>(2) * sms, p.B));
-    if (launch_dependent(k_decide<Tag, MODE>, blocksd, decide_smem(p.R), st, p, kDecideThreads) != SPEC_OK)
+    if (launch_dependent(k_decide<Tag, MODE>, blocksd, decide_smem(p.R, p.S), st, p, kDecideThreads) != SPEC_OK)
         return SPEC_ECUDA;
     if (p.nP == 0) return SPEC_OK;
 
@@ -255,10 +275,12 @@ int launch_verify(Params &p, const Layout &L, void *ws, int dtype_index, cudaStr
     return launch_dependent(k_finalize<Tag, MODE>, blocks3, dyn3, st, p);
 }
 
-// The one-kernel linear path: clear the counters, then one resident wave.
+// The one-kernel linear path: one cooperative launch (the kernel clears its
+// own counters before a grid-wide barrier), exactly one resident wave.  A
+// grid that cannot be resident at once fails to launch (SPEC_ECUDA).
 int g_fused_blocks[64][2];
 template <class Tag>
-int launch_fused(Params &p, const Layout &L, void *ws, int dtype_index, cudaStream_t st)
+int launch_fused(Params &p, int dtype_index, cudaStream_t st)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SPEC_ECUDA;
@@ -272,12 +294,84 @@ int launch_fused(Params &p, const Layout &L, void *ws, int dtype_index, cudaStre
     // whole static rounds for about the first 88% of the pass-1 items
     const unsigned W = static_cast<unsigned>(per_sm * sms * kStreamers);
     p.nAs = static_cast<unsigned>((static_cast<uint64_t>(p.nA) * 88 / 100) / W * W);
-    // counters and pass-1 partials to all ones (kPartEmpty), one contiguous range
-    const size_t clear = L.rowpart - L.counters + sizeof(float2) * static_cast<size_t>(p.nA);
-    if (cudaMemsetAsync(static_cast<char *>(ws) + L.counters, 0xFF, clear, st) != cudaSuccess)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(per_sm * sms));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kFusedSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k_fused<Tag>, p) != cudaSuccess) {
+        (void)cudaGetLastError();  // the error is returned, not left for the next call
         return SPEC_ECUDA;
-    k_fused<Tag><<<static_cast<unsigned>(per_sm * sms), kThreads, kFusedSmem, st>>>(p);
-    return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ECUDA;
+    }
+    return SPEC_OK;
+}
+
+// The distribution-exact tree mode: pass 1 as the independent-test mode,
+// then the cluster kernel k_tree_exact (one cluster per request, up to the
+// co-resident maximum), a programmatic dependent of pass 1.
+int g_exact_clusters[64][2];
+template <class Tag>
+int launch_exact(Params &p, int dtype_index, cudaStream_t st)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SPEC_ECUDA;
+    int per_sm1, sms, maxc;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        per_sm1 = blocks_per_sm(g_pass1_blocks[dev][dtype_index][kTreeStochastic],
+                                k_pass1<Tag, kTreeStochastic, 2>, kRingBytes);
+        sms = sm_count(dev);
+        int &slot = g_exact_clusters[dev][dtype_index];
+        if (slot < 1) {
+            cudaLaunchConfig_t q = {};
+            cudaLaunchAttribute qa[1];
+            qa[0].id = cudaLaunchAttributeClusterDimension;
+            qa[0].val.clusterDim.x = kExactCluster;
+            qa[0].val.clusterDim.y = 1;
+            qa[0].val.clusterDim.z = 1;
+            q.gridDim = dim3(kExactCluster);
+            q.blockDim = dim3(kThreads);
+            q.attrs = qa;
+            q.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, k_tree_exact<Tag, kExactCluster>, &q) != cudaSuccess || n < 1)
+                return SPEC_ECUDA;
+            slot = n;
+        }
+        maxc = slot;
+    }
+    if (per_sm1 < 1 || sms < 1 || maxc < 1) return SPEC_ECUDA;
+    const int64_t blocks1 =
+        std::max<int64_t>(1, std::min<int64_t>(static_cast<int64_t>(per_sm1) * sms, ceil_div(p.nA, kWarps)));
+    k_pass1<Tag, kTreeStochastic, 2><<<static_cast<unsigned>(blocks1), kThreads, kRingBytes, st>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return SPEC_ECUDA;
+    const int ncl = std::min(maxc, p.B);
+    const int slice = static_cast<int>(ceil_div(ceil_div(p.V, kExactCluster), Tag::kVec) * Tag::kVec);
+    const int chunk = static_cast<int>(ceil_div(ceil_div(slice, kThreads), Tag::kVec) * Tag::kVec);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kExactCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(ncl) * kExactCluster);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, k_tree_exact<Tag, kExactCluster>, p, slice, chunk) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return SPEC_ECUDA;
+    }
+    return SPEC_OK;
 }
 
 // Largest number of co-resident greedy clusters, per device and dtype.
@@ -353,6 +447,7 @@ void base_params(Params &p, const void *tl, const void *dl, int64_t stride, int 
     p.offset = offset;
     p.S2 = static_cast<int>(ceil_div(V, kSeg2));
     p.W32 = p.S2 * (kSeg2 / 32);
+    p.poll_limit = kWaitPolls;
     fill_exp2_table(p);
 }
 
@@ -369,6 +464,8 @@ int setup_items(Params &p, int R, spec_dtype_t dtype, bool pass2)
     p.div_req = make_fastdiv(static_cast<uint32_t>(R) * static_cast<uint32_t>(p.S));
     p.div_s = make_fastdiv(static_cast<uint32_t>(p.S));
     p.div_s2 = make_fastdiv(static_cast<uint32_t>(p.S2));
+    const int chunk = dtype == SPEC_BF16 ? kP2ChunkBf16 : kP2ChunkF32;
+    p.div_cpr = make_fastdiv(static_cast<uint32_t>((p.S2 + chunk - 1) / chunk));
     return SPEC_OK;
 }
 
@@ -396,13 +493,16 @@ extern "C" const char *spec_verify_strerror(int code)
     }
 }
 
-extern "C" int spec_verify_linear(const void *target_logits, const void *draft_logits,
-                                  spec_dtype_t dtype, int64_t row_stride,
-                                  const int32_t *draft_tokens, int batch, int k, int vocab,
-                                  float temperature, uint64_t seed, uint32_t offset,
-                                  int32_t *out_tokens, int32_t *accepted_len, float *dbg_logp,
-                                  float *dbg_logq, int32_t *status, void *workspace,
-                                  size_t workspace_bytes, cudaStream_t stream)
+namespace {
+
+// spec_verify_linear, with the diagnostic switches of
+// spec_verify_debug_wait_expiry (poll_limit 0: the normal limit).
+int linear_call(const void *target_logits, const void *draft_logits, spec_dtype_t dtype,
+                int64_t row_stride, const int32_t *draft_tokens, int batch, int k, int vocab,
+                float temperature, uint64_t seed, uint32_t offset, int32_t *out_tokens,
+                int32_t *accepted_len, float *dbg_logp, float *dbg_logq, int32_t *status,
+                void *workspace, size_t workspace_bytes, cudaStream_t stream, bool diag,
+                unsigned poll_limit)
 {
     if (batch < 0 || k < 1) return SPEC_EINVAL;
     if (k > SPEC_MAX_K) return SPEC_EUNSUPPORTED;
@@ -430,11 +530,44 @@ extern "C" int spec_verify_linear(const void *target_logits, const void *draft_l
     p.dbg_lp = dbg_logp;
     p.dbg_lq = dbg_logq;
     p.status = status;
+    if (diag) {
+        p.diag_no_partials = 1;
+        p.poll_limit = poll_limit;
+    }
     rc = setup_items(p, R, dtype, true);
     if (rc != SPEC_OK) return rc;
     fill_workspace(p, workspace, L);
-    return dtype == SPEC_BF16 ? launch_fused<Bf16>(p, L, workspace, 1, stream)
-                              : launch_fused<F32>(p, L, workspace, 0, stream);
+    return dtype == SPEC_BF16 ? launch_fused<Bf16>(p, 1, stream) : launch_fused<F32>(p, 0, stream);
+}
+
+}  // namespace
+
+extern "C" int spec_verify_linear(const void *target_logits, const void *draft_logits,
+                                  spec_dtype_t dtype, int64_t row_stride,
+                                  const int32_t *draft_tokens, int batch, int k, int vocab,
+                                  float temperature, uint64_t seed, uint32_t offset,
+                                  int32_t *out_tokens, int32_t *accepted_len, float *dbg_logp,
+                                  float *dbg_logq, int32_t *status, void *workspace,
+                                  size_t workspace_bytes, cudaStream_t stream)
+{
+    return linear_call(target_logits, draft_logits, dtype, row_stride, draft_tokens, batch, k,
+                       vocab, temperature, seed, offset, out_tokens, accepted_len, dbg_logp,
+                       dbg_logq, status, workspace, workspace_bytes, stream, false, 0);
+}
+
+extern "C" int spec_verify_debug_wait_expiry(const void *target_logits, const void *draft_logits,
+                                             spec_dtype_t dtype, int64_t row_stride,
+                                             const int32_t *draft_tokens, int batch, int k,
+                                             int vocab, float temperature, uint32_t poll_limit,
+                                             int32_t *out_tokens, int32_t *accepted_len,
+                                             int32_t *status, void *workspace,
+                                             size_t workspace_bytes, cudaStream_t stream)
+{
+    if (poll_limit < 1 || poll_limit > SPEC_DEBUG_MAX_POLLS) return SPEC_EINVAL;
+    if (!status) return SPEC_EINVAL;
+    return linear_call(target_logits, draft_logits, dtype, row_stride, draft_tokens, batch, k,
+                       vocab, temperature, 0, 0, out_tokens, accepted_len, nullptr, nullptr,
+                       status, workspace, workspace_bytes, stream, true, poll_limit);
 }
 
 extern "C" int spec_verify_greedy(const void *target_logits, spec_dtype_t dtype,
@@ -471,6 +604,7 @@ extern "C" int spec_verify_tree(const void *target_logits, const void *draft_log
 {
     if (batch < 0 || num_nodes < 1 || max_depth < 1) return SPEC_EINVAL;
     if (num_nodes > SPEC_MAX_NODES) return SPEC_EUNSUPPORTED;
+    if (stochastic < 0 || stochastic > 2) return SPEC_EINVAL;
     if (stochastic && (!(temperature > 0.f) || !(temperature < INFINITY))) return SPEC_EINVAL;
     int rc = check_shape(dtype, row_stride, vocab);
     if (rc != SPEC_OK) return rc;
@@ -497,9 +631,11 @@ extern "C" int spec_verify_tree(const void *target_logits, const void *draft_log
     p.acc = accepted_len;
     p.path = out_path_nodes;
     p.status = status;
-    rc = setup_items(p, R, dtype, stochastic != 0);
+    rc = setup_items(p, R, dtype, stochastic == 1);
     if (rc != SPEC_OK) return rc;
     fill_workspace(p, workspace, L);
+    if (stochastic == 2)
+        return dtype == SPEC_BF16 ? launch_exact<Bf16>(p, 1, stream) : launch_exact<F32>(p, 0, stream);
     if (dtype == SPEC_BF16)
         return stochastic ? launch_verify<Bf16, kTreeStochastic>(p, L, workspace, 1, stream)
                           : launch_verify<Bf16, kTreeGreedy>(p, L, workspace, 1, stream);

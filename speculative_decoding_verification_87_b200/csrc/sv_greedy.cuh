@@ -10,8 +10,10 @@
 // lowest argmax, NaN seen) in its shared memory; after a cluster barrier the
 // rank-0 block merges the CL partials through distributed shared memory,
 // scans for the first mismatch and writes the outputs.  Partials are double
-// buffered, so one barrier per request suffices.  Clusters stride over the
-// batch; a block's reads run one step ahead of its reductions and barriers.
+// buffered and the cluster barrier is split (arrive, then wait): only rank 0
+// waits at the end of a request, the other blocks go on to the next one.
+// Clusters stride over the batch; a block's reads run one step ahead of its
+// reductions and barriers.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -22,6 +24,18 @@
 namespace sv {
 
 constexpr int kMaxRowsGreedy = 33;  // k + 1 with k <= 32
+
+// Split cluster barrier (all threads of every block of the cluster, in
+// step): arrive with release semantics, wait with acquire semantics; a
+// thread waits for a phase before it arrives for the next one.
+__device__ __forceinline__ void cluster_arrive()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait()
+{
+    asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
 
 template <class Tag, int CL>
 __global__ void __launch_bounds__(kThreads) k_greedy_cluster(const Params p, int slice)
@@ -34,8 +48,7 @@ __global__ void __launch_bounds__(kThreads) k_greedy_cluster(const Params p, int
     constexpr int kChunk = kThreads * kVec * U;  // entries of a slice read per step
 
     __shared__ float2 part[2][kMaxRowsGreedy];
-    __shared__ float redf[kWarps];
-    __shared__ int redi[kWarps];
+    __shared__ float2 wpart[2][kMaxRowsGreedy][kWarps];
     __shared__ int g_sh[kMaxRowsGreedy];
     __shared__ int nan_sh;
 
@@ -81,23 +94,32 @@ __global__ void __launch_bounds__(kThreads) k_greedy_cluster(const Params p, int
         }
         if (nb < p.B) load(nb, nj, nit, nxt);
         const int base = s_begin + it * kChunk;
+        // a thread visits its entries in increasing index order, so a later
+        // entry equal to the running max never replaces it (ties go to the
+        // lowest index); a vector's packed max decides whether any entry of
+        // it can matter, and only then are its entries searched
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int e0 = base + (tid + u * kThreads) * kVec;
             uint4 raw = cur[u];
             if (e0 < s_end && e0 + kVec > s_end) raw = mask_tail<Tag>(raw, s_end - e0);
-            float x[kVec];
-            unpack<Tag>(raw, x);
+            const float vm = vec_max<Tag>(raw);  // NaN if any entry is NaN
+            if (!(vm <= best)) {
+                if (vm != vm) {
+                    nan = true;
+                } else {
+                    float x[kVec];
+                    unpack<Tag>(raw, x);
+                    int first = kVec - 1;
 #pragma unroll
-            for (int e = 0; e < kVec; ++e) {
-                nan |= (x[e] != x[e]);
-                if (x[e] > best) {
-                    best = x[e];
-                    idx = e0 + e;
+                    for (int e = kVec - 1; e >= 0; --e)
+                        if (x[e] == vm) first = e;
+                    best = vm;
+                    idx = e0 + first;
                 }
             }
         }
-        if (it == iters - 1) {  // row j of request b is reduced: merge the block
+        if (it == iters - 1) {  // row j of request b is reduced in this block
             const int buf = rq & 1;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
@@ -105,25 +127,32 @@ __global__ void __launch_bounds__(kThreads) k_greedy_cluster(const Params p, int
                 const int oi = __shfl_xor_sync(kFull, idx, o);
                 argmax_take(best, idx, ov, oi);
             }
-            const int any_nan = __syncthreads_or(nan ? 1 : 0);
-            if (lane == 0) {
-                redf[warp] = best;
-                redi[warp] = idx;
-            }
-            __syncthreads();
-            if (tid == 0) {
-                float bv = redf[0];
-                int bi = redi[0];
-                for (int w = 1; w < kWarps; ++w) argmax_take(bv, bi, redf[w], redi[w]);
-                part[buf][j] = make_float2(any_nan ? __int_as_float(0x7FC00000) : bv, __int_as_float(bi));
-            }
-            __syncthreads();
+            nan = __any_sync(kFull, nan);
+            if (lane == 0) wpart[buf][j][warp] = make_float2(nan ? __int_as_float(0x7FC00000) : best, __int_as_float(idx));
             best = -INFINITY;
             idx = INT_MAX;
             nan = false;
-            if (j == k) {  // the request is reduced in every block of the cluster
-                cluster.sync();
+            if (j == k) {  // the request is reduced in every warp of the block
+                __syncthreads();
+                for (int jj = tid; jj <= k; jj += kThreads) {
+                    float bv = -INFINITY;
+                    int bi = INT_MAX;
+                    bool nn = false;
+#pragma unroll
+                    for (int w = 0; w < kWarps; ++w) {
+                        const float2 v = wpart[buf][jj][w];
+                        if (v.x != v.x) nn = true;
+                        else argmax_take(bv, bi, v.x, __float_as_int(v.y));
+                    }
+                    part[buf][jj] = make_float2(nn ? __int_as_float(0x7FC00000) : bv, __int_as_float(bi));
+                }
+                // split cluster barrier: every block arrives once its partials
+                // are in place; only rank 0 waits here (it reads them all), the
+                // others wait for this phase just before their next arrival
+                if (rq > 0 && rank != 0) cluster_wait();
+                cluster_arrive();
                 if (rank == 0) {
+                    cluster_wait();
                     if (tid == 0) nan_sh = 0;
                     __syncthreads();
                     for (int jj = tid; jj <= k; jj += kThreads) {
@@ -171,7 +200,11 @@ __global__ void __launch_bounds__(kThreads) k_greedy_cluster(const Params p, int
         j = nj;
         it = nit;
     }
-    cluster.sync();  // no block leaves while rank 0 may still read its partials
+    // the last phase: rank 0 has waited on it; the others wait now, then one
+    // full barrier so that no block leaves while rank 0 may still read its
+    // partials
+    if (rq > 0 && rank != 0) cluster_wait();
+    cluster.sync();
 }
 
 }  // namespace sv

@@ -63,6 +63,11 @@ struct TreeScratch {
     short depth[kMaxNodes];
     unsigned char flag[kMaxNodes];  // 1 has child, 2 test passed, 4 accepted
 };
+// The logits a stochastic tree's node tests read (target and draft row of
+// the parent at the node's token), fetched before pass 1 completes.
+struct TreeProbe {
+    float lt[kMaxNodes], ld[kMaxNodes];
+};
 
 // ------------------------------------------------------------ small helpers
 
@@ -365,7 +370,7 @@ __device__ __forceinline__ void reduce_item1(const Params &p, unsigned item, int
         sr = warp_sum(sr);
         part = make_float2(M, sr);
     }
-    if (lane == 0) __stcg(p.rowpart + item, part);
+    if (lane == 0 && !p.diag_no_partials) __stcg(p.rowpart + item, part);
 }
 
 // The pass-1 worker: warp w of W takes items w, w + W, w + 2W, ... (items
@@ -422,16 +427,19 @@ struct RowStats {
 // partial sums rescaled on the FMA pipe and accumulated in fp64.  Greedy
 // rows: (max, lowest argmax).  One warp; fixed order, so deterministic.
 template <int MODE>
-__device__ __forceinline__ void merge_row(const Params &p, int b, int r, RowStats rs)
+__device__ __forceinline__ void merge_row(const Params &p, int b, int r, RowStats rs,
+                                          const float2 *staged = nullptr)
 {
     const int lane = threadIdx.x & 31;
-    const float2 *part = p.rowpart + (static_cast<int64_t>(b) * p.R + r) * p.S;
+    // the row's partials: in global memory, or staged in shared memory
+    const float2 *part = staged ? staged + static_cast<int64_t>(r) * p.S
+                                : p.rowpart + (static_cast<int64_t>(b) * p.R + r) * p.S;
     if (MODE == kTreeGreedy) {
         float bv = -INFINITY;
         int bi = INT_MAX;
         bool nan = false;
         for (int sg = lane; sg < p.S; sg += 32) {
-            const float2 v = __ldcg(part + sg);
+            const float2 v = staged ? part[sg] : __ldcg(part + sg);
             if (v.x != v.x) nan = true;
             else if (v.x != -INFINITY) argmax_take(bv, bi, v.x, __float_as_int(v.y));
         }
@@ -452,7 +460,7 @@ __device__ __forceinline__ void merge_row(const Params &p, int b, int r, RowStat
         double s = 0.0;
         bool nan = false;
         for (int sg = lane; sg < p.S; sg += 32) {
-            const float2 v = __ldcg(part + sg);
+            const float2 v = staged ? part[sg] : __ldcg(part + sg);
             if (v.x != v.x || v.y != v.y) {
                 nan = true;
             } else if (v.x > m) {
@@ -571,8 +579,14 @@ __device__ __forceinline__ void decide_linear(const Params &p, int b, RowStats s
 }
 
 
+// The tree decide step of request b, one warp: checks, node tests (lanes
+// over nodes; stochastic tests read the prefetched logits), then depths and
+// acceptance level by level (at most max_depth + 1 rounds, lanes over
+// nodes), the deepest accepted node by a warp reduction (ties to the
+// lowest index), and the outputs.
 template <class Tag, int MODE>
-__device__ __forceinline__ void decide_tree(const Params &p, int b, RowStats rs, TreeScratch &sh)
+__device__ __forceinline__ void decide_tree(const Params &p, int b, RowStats rs, TreeScratch &sh,
+                                            const TreeProbe *pr)
 {
     const int lane = threadIdx.x & 31;
     const int N = p.N, R = p.R;
@@ -581,6 +595,7 @@ __device__ __forceinline__ void decide_tree(const Params &p, int b, RowStats rs,
     int err = 0;  // sh.flag holds "has a child" (bit 1), set by the block
     for (int i = lane; i < N; i += 32) {
         const int par = __ldg(pa + i);
+        sh.depth[i] = i == 0 ? 0 : -1;
         if (i == 0) {
             if (par != -1) err |= kStTree;
         } else if (par < 0 || par >= i) {
@@ -593,16 +608,21 @@ __device__ __forceinline__ void decide_tree(const Params &p, int b, RowStats rs,
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) err |= __shfl_xor_sync(kFull, err, o);
     __syncwarp();
-    if (lane == 0 && !(err & kStTree)) {
-        sh.depth[0] = 0;
-        for (int i = 1; i < N; ++i) {
-            const int d = sh.depth[__ldg(pa + i)] + 1;
-            sh.depth[i] = static_cast<short>(d);
-            if (d > p.max_depth) err |= kStTree;
+    if (!(err & kStTree)) {
+        // depth of every node: its parent's plus one, settled one level per
+        // round; a node still unset after max_depth + 1 rounds is too deep
+        for (int round = 0; round <= p.max_depth; ++round) {
+            for (int i = 1 + lane; i < N; i += 32) {
+                if (sh.depth[i] >= 0) continue;
+                const int dp = sh.depth[__ldg(pa + i)];
+                if (dp >= 0) sh.depth[i] = static_cast<short>(dp + 1);
+            }
+            __syncwarp();
         }
+        bool deep = false;
+        for (int i = lane; i < N; i += 32) deep |= sh.depth[i] < 0 || sh.depth[i] > p.max_depth;
+        if (__any_sync(kFull, deep)) err |= kStTree;
     }
-    err = __shfl_sync(kFull, err, 0);
-    __syncwarp();
 
     // rows the mode reads must be usable: every target row, and the draft
     // rows of nodes with children
@@ -620,11 +640,10 @@ __device__ __forceinline__ void decide_tree(const Params &p, int b, RowStats rs,
             if (MODE == kTreeGreedy) {
                 ok = (t == rs.idx[par]);
             } else {
-                const int64_t off = (static_cast<int64_t>(b) * N + par) * p.stride + t;
                 const double lp =
-                    (logit_f64_at<Tag>(p.tl, off) - static_cast<double>(rs.m[par])) * p.inv_t - log(rs.s[par]);
-                const double lq = (logit_f64_at<Tag>(p.dl, off) - static_cast<double>(rs.m[N + par])) * p.inv_t -
-                                  log(rs.s[N + par]);
+                    (f32_to_f64(pr->lt[i]) - static_cast<double>(rs.m[par])) * p.inv_t - log(rs.s[par]);
+                const double lq =
+                    (f32_to_f64(pr->ld[i]) - static_cast<double>(rs.m[N + par])) * p.inv_t - log(rs.s[N + par]);
                 const double u = philox_uniform(p.seed, static_cast<uint32_t>(b),
                                                 static_cast<uint32_t>(i - 1), kPurposeAccept, p.offset);
                 ok = accept_test(lp, lq, u);
@@ -633,32 +652,44 @@ __device__ __forceinline__ void decide_tree(const Params &p, int b, RowStats rs,
         }
     }
     __syncwarp();
-    if (lane != 0) return;
 
     const int W = p.max_depth + 1;
     int32_t *out = p.out + static_cast<int64_t>(b) * W;
     int32_t *path = p.path ? p.path + static_cast<int64_t>(b) * W : nullptr;
-    for (int j = 0; j < W; ++j) {
+    ReqInfo info = empty_req();
+    if (err) {
+        for (int j = lane; j < W; j += 32) {
+            out[j] = -1;
+            if (path) path[j] = -1;
+        }
+        if (lane == 0) {
+            p.acc[b] = -1;
+            report(p.status, err);
+            store_req(p.req + b, info);
+        }
+        return;
+    }
+    // acceptance level by level: a node is accepted when its parent is and
+    // its test passed; the deepest accepted node wins, ties to the lowest index
+    if (lane == 0) sh.flag[0] |= 4;
+    __syncwarp();
+    for (int lvl = 1; lvl <= p.max_depth; ++lvl) {
+        for (int i = 1 + lane; i < N; i += 32)
+            if (sh.depth[i] == lvl && (sh.flag[__ldg(pa + i)] & 4) && (sh.flag[i] & 2)) sh.flag[i] |= 4;
+        __syncwarp();
+    }
+    int key = 0;  // depth << 11 | (kMaxNodes - 1 - node): larger is deeper, then lower index
+    for (int i = lane; i < N; i += 32)
+        if (sh.flag[i] & 4) key = max(key, (static_cast<int>(sh.depth[i]) << 11) | (kMaxNodes - 1 - i));
+    key = warp_max(key);
+    const int d = kMaxNodes - 1 - (key & 2047);
+    const int D = sh.depth[d];
+    for (int j = lane; j < W; j += 32) {
         out[j] = -1;
         if (path) path[j] = -1;
     }
-    ReqInfo info = empty_req();
-    if (err) {
-        p.acc[b] = -1;
-        report(p.status, err);
-        store_req(p.req + b, info);
-        return;
-    }
-    sh.flag[0] |= 4;
-    int d = 0;
-    for (int i = 1; i < N; ++i) {
-        const bool a = (sh.flag[__ldg(pa + i)] & 4) && (sh.flag[i] & 2);
-        if (a) {
-            sh.flag[i] |= 4;
-            if (sh.depth[i] > sh.depth[d]) d = i;
-        }
-    }
-    const int D = sh.depth[d];
+    __syncwarp();
+    if (lane != 0) return;
     for (int node = d; node != 0; node = __ldg(pa + node)) {
         out[sh.depth[node] - 1] = __ldg(tk + node);
         if (path) path[sh.depth[node]] = node;
@@ -1187,20 +1218,44 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) k_pass1(const __grid_con
 // at once for up to 32) into shared memory, then warp 0 runs the decide
 // step.
 constexpr int kDecideThreads = 1024;
+// partials a decide block stages in shared memory (beyond that it reads them
+// through L2): 12288 x 8 B = 96 KB
+constexpr int kDecideStageMax = 12288;
 template <class Tag, int MODE>
 __global__ void __launch_bounds__(kDecideThreads) k_decide(const __grid_constant__ Params p)
 {
     constexpr int kDW = kDecideThreads / 32;
     extern __shared__ double rowmem[];
     __shared__ TreeScratch ts;
+    __shared__ TreeProbe tp;
     const int warp = threadIdx.x >> 5;
     RowStats rs;
     rs.s = rowmem;
     rs.m = reinterpret_cast<float *>(rowmem + p.R);
     rs.idx = reinterpret_cast<int *>(rs.m + p.R);
+    const bool stage_parts = p.R * p.S <= kDecideStageMax;
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
     DraftProbe pr;
     if (MODE == kLinear && warp == 0) pr = probe_drafts<Tag>(p, blockIdx.x);
+    // stochastic trees: the logits each node test reads are inputs, fetched
+    // before pass 1 completes (a thread per node)
+    auto fetch_tests = [&](int b) {
+        if (MODE != kTreeStochastic || b >= p.B) return;
+        const int32_t *pa = p.parents + static_cast<int64_t>(b) * p.N;
+        const int32_t *tk = p.tokens + static_cast<int64_t>(b) * p.N;
+        for (int i = 1 + threadIdx.x; i < p.N; i += kDecideThreads) {
+            const int par = __ldg(pa + i), t = __ldg(tk + i);
+            float lt = 0.f, ld = 0.f;
+            if (par >= 0 && par < i && t >= 0 && t < p.V) {
+                const int64_t off = (static_cast<int64_t>(b) * p.N + par) * p.stride + t;
+                lt = load_logit<Tag>(p.tl, off);
+                ld = load_logit<Tag>(p.dl, off);
+            }
+            tp.lt[i] = lt;
+            tp.ld[i] = ld;
+        }
+    };
+    fetch_tests(blockIdx.x);
     asm volatile("griddepcontrol.wait;\n" ::: "memory");
     for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
         if (MODE != kLinear) {
@@ -1214,9 +1269,19 @@ __global__ void __launch_bounds__(kDecideThreads) k_decide(const __grid_constant
             }
             __syncthreads();
         }
+        // the request's partials, staged in shared memory by every thread at
+        // once (one round of independent loads) when they fit, then merged
+        // a warp per row
+        float2 *stg = stage_parts ? reinterpret_cast<float2 *>(rs.idx + p.R) : nullptr;
+        if (stage_parts) {
+            const float2 *src = p.rowpart + static_cast<int64_t>(b) * p.R * p.S;
+            const int n = p.R * p.S;
+            for (int i = threadIdx.x; i < n; i += kDecideThreads) stg[i] = __ldcg(src + i);
+            __syncthreads();
+        }
         for (int r = warp; r < p.R; r += kDW) {
             if (MODE != kLinear && r >= p.N && !ts.flag[r - p.N]) continue;
-            merge_row<MODE>(p, b, r, rs);
+            merge_row<MODE>(p, b, r, rs, stg);
         }
         __syncthreads();
         if (warp == 0) {
@@ -1224,10 +1289,14 @@ __global__ void __launch_bounds__(kDecideThreads) k_decide(const __grid_constant
                 decide_linear<Tag>(p, b, rs, pr);
                 pr = probe_drafts<Tag>(p, b + gridDim.x);
             } else {
-                decide_tree<Tag, MODE>(p, b, rs, ts);
+                decide_tree<Tag, MODE>(p, b, rs, ts, &tp);
             }
         }
         __syncthreads();
+        if (b + static_cast<int>(gridDim.x) < p.B) {
+            fetch_tests(b + gridDim.x);
+            __syncthreads();
+        }
     }
 }
 
@@ -1237,9 +1306,9 @@ template <class Tag, int MODE>
 __global__ void __launch_bounds__(kThreads, 3) k_pass2(const __grid_constant__ Params p)
 {
     extern __shared__ uint4 dyn[];
-    __shared__ double tab[64];
+    __shared__ double tab[kExp2Tab];
     const int warp = threadIdx.x >> 5;
-    if (threadIdx.x < 64) tab[threadIdx.x] = p.exp2tab[threadIdx.x];
+    for (int j = threadIdx.x; j < kExp2Tab; j += kThreads) tab[j] = p.exp2tab[j];
     __syncthreads();
     uint4 *stage = dyn + warp * StageShape<Tag>::kPerWarp;
     // the finalize grid may be scheduled as blocks of this one retire
@@ -1303,9 +1372,9 @@ template <class Tag, int MODE>
 __global__ void __launch_bounds__(kThreads) k_finalize(const __grid_constant__ Params p)
 {
     extern __shared__ double wdyn[];
-    __shared__ double tab[64];
+    __shared__ double tab[kExp2Tab];
     const int warp = threadIdx.x >> 5;
-    if (threadIdx.x < 64) tab[threadIdx.x] = p.exp2tab[threadIdx.x];
+    for (int j = threadIdx.x; j < kExp2Tab; j += kThreads) tab[j] = p.exp2tab[j];
     __syncthreads();
     const bool w_shared = p.S2 <= kMaxS2Shared;
     asm volatile("griddepcontrol.wait;\n" ::: "memory");

@@ -85,6 +85,53 @@ def test_linear_host_validation(lib):
     assert _linear(lib, batch=0, tl=0, dl=0, tokens=0) == SPEC_OK
 
 
+def test_noalloc_checks_arguments_before_the_scratch_size(lib):
+    # too large for the static scratch: SPEC_EUNSUPPORTED, unless an argument
+    # is invalid, which keeps the code spec_verify_linear gives it
+    P = ctypes.c_void_p
+
+    def na(**kw):
+        return lib.spec_verify_linear_noalloc(
+            P(kw.get("tl", 0x1000)), P(0x2000), 1, 128256, P(0x3000), kw.get("batch", 5000), 8,
+            128256, kw.get("temp", 1.0), 0, 0, P(0x4000), P(0x5000), None, None, None, None)
+    assert na() == SPEC_EUNSUPPORTED
+    assert na(temp=0.0) == SPEC_EINVAL
+    assert na(tl=0) == SPEC_EINVAL
+    assert na(tl=0x1008) == SPEC_EALIGN
+
+
+def test_debug_wait_expiry_host_validation(lib):
+    P = ctypes.c_void_p
+
+    def d(**kw):
+        return lib.spec_verify_debug_wait_expiry(
+            P(0x1000), P(0x2000), 1, 128, P(0x3000), 2, 3, 100, 1.0, kw.get("polls", 16),
+            P(0x4000), P(0x5000), P(kw.get("status", 0x6000)), P(kw.get("ws", 0x10000)),
+            kw.get("ws_bytes", 1 << 30), None)
+    assert d(polls=0) == SPEC_EINVAL
+    assert d(polls=4097) == SPEC_EINVAL
+    assert d(status=0) == SPEC_EINVAL     # the expiry is reported through status
+    assert d(ws=0) == SPEC_EWORKSPACE
+
+
+def test_plug_host_validation(lib):
+    P = ctypes.c_void_p
+
+    def pl(**kw):
+        return lib.spec_plug_tokens(P(kw.get("inp", 0x1000)), P(kw.get("out", 0x2000)),
+                                    P(kw.get("acc", 0x3000)), kw.get("batch", 4), kw.get("k", 3),
+                                    P(kw.get("nxt", 0x4000)), P(kw.get("seq", 0)),
+                                    P(kw.get("ln", 0)), kw.get("cap", 0), None, None)
+    assert pl(k=0) == SPEC_EINVAL and pl(k=33) == SPEC_EUNSUPPORTED
+    assert pl(batch=-1) == SPEC_EINVAL and pl(cap=-1) == SPEC_EINVAL
+    assert pl(seq=0x5000) == SPEC_EINVAL          # seq_tokens without seq_len
+    assert pl(ln=0x5000) == SPEC_EINVAL           # seq_len without seq_tokens
+    assert pl(out=0) == SPEC_EINVAL and pl(acc=0) == SPEC_EINVAL
+    assert pl(inp=0) == SPEC_EINVAL               # next_tokens needs the inputs
+    assert pl(nxt=0) == SPEC_OK                   # nothing asked for: nothing enqueued
+    assert pl(batch=0, out=0, acc=0) == SPEC_OK
+
+
 def test_greedy_and_tree_host_validation(lib):
     P = ctypes.c_void_p
     g = lambda **kw: lib.spec_verify_greedy(P(kw.get("tl", 0x1000)), kw.get("dtype", 0),
@@ -106,6 +153,8 @@ def test_greedy_and_tree_host_validation(lib):
     assert t(dl=0) == SPEC_EINVAL                 # stochastic trees read draft rows
     assert t(dl=0, batch=0) == SPEC_OK            # an empty batch reads nothing
     assert t(temp=-1.0) == SPEC_EINVAL
+    assert t(stoch=3) == SPEC_EINVAL and t(stoch=-1) == SPEC_EINVAL
+    assert t(stoch=2, dl=0) == SPEC_EINVAL        # the exact mode reads draft rows too
     assert t(ws_bytes=8) == SPEC_EWORKSPACE
     assert t(batch=0) == SPEC_OK
 

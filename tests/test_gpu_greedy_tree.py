@@ -4,7 +4,7 @@ import pytest
 import torch
 
 from speculative_decoding_verification_87_b200 import workloads as wl
-from parity import compare_tree_stochastic, to_device
+from parity import FlagTally, TreeOnDevice, compare_tree_stochastic, oracle_tree_many, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -104,14 +104,19 @@ def test_tree_greedy_full_size_bit_exact(sv, orc):
 
 
 def test_tree_stochastic_full_size(sv, orc):
+    """B=32, N=60, depth 6, V=128256 bf16, T=1 at 200 offsets: 6400
+    requests of 60 trials each (59 node tests and one draw)."""
     w = wl.config_tree(seed=0)
-    for off in range(3):
-        out, acc, path, st = run_tree(sv, w, True, seed=5, offset=off)
-        o = orc.verify_tree(w.target, w.draft, w.node_tokens, w.parents, w.max_depth, w.vocab,
-                            True, w.temperature, 5, off)
-        assert st == 0
-        r = compare_tree_stochastic(out, acc, path, o)
-        print("tree stochastic", r, "mean depth", acc.mean())
+    offsets = range(200)
+    gpu = TreeOnDevice(sv, w).run_many(True, 5, offsets)
+    orcs = oracle_tree_many(orc, w, True, 5, offsets)
+    tally = FlagTally()
+    depths = []
+    for g, o in zip(gpu, orcs):
+        assert g["status"] == 0
+        tally.add(compare_tree_stochastic(g["out"], g["acc"], g["path"], o))
+        depths.extend(g["acc"].tolist())
+    print("tree stochastic", tally.check(min_trials=100_000), "mean depth", np.mean(depths))
 
 
 def test_chain_tree_equals_linear_greedy_on_gpu(sv):
@@ -154,6 +159,7 @@ def test_tree_errors(sv, orc):
 
 
 def test_small_trees_both_modes(sv, orc):
+    tally = FlagTally()
     for seed in range(4):
         w = wl.draft_tree(seed=seed, batch=16, vocab=777, level_widths=(1, 3, 4, 2), topk=3,
                           dtype="f32", pad=3)
@@ -163,6 +169,7 @@ def test_small_trees_both_modes(sv, orc):
                                 w.vocab, stochastic, 1.0, seed, 1)
             assert st == 0
             if stochastic:
-                compare_tree_stochastic(out, acc, path, o)
+                tally.add(compare_tree_stochastic(out, acc, path, o))
             else:
                 assert np.array_equal(out, o["out"]) and np.array_equal(path, o["path"])
+    tally.check()

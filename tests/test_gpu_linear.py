@@ -4,8 +4,9 @@ import pytest
 import torch
 
 from speculative_decoding_verification_87_b200 import workloads as wl
-from parity import compare_linear, run_linear_gpu, to_device
-from stats_util import chisquare_pvalue, softmax64
+from parity import (FlagTally, LinearOnDevice, compare_linear, oracle_linear_many, run_linear_gpu,
+                    to_device)
+from stats_util import brute_force_linear, chisquare_pvalue, softmax64
 
 pytestmark = pytest.mark.gpu
 
@@ -29,11 +30,13 @@ def test_device_philox_matches_oracle(sv, orc):
 
 def test_tiny_config_matches_oracle(sv, orc):
     w = wl.config_tiny(seed=0)
+    tally = FlagTally()
     for off in range(50):
         g = run_linear_gpu(sv, w, seed=0, offset=off)
         o = orc.verify_linear(w.target, w.draft, w.tokens, w.vocab, w.temperature, 0, off)
         assert g["status"] == 0
-        compare_linear(g, o, w.k)
+        tally.add(compare_linear(g, o, w.k))
+    tally.check()
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
@@ -48,21 +51,25 @@ def test_ragged_vocab_and_stride(sv, orc, dtype, vocab, pad):
         t[..., vocab:] = nan
         d[..., vocab:] = nan
     w.target, w.draft = t, d
+    tally = FlagTally()
     for off in range(8):
         g = run_linear_gpu(sv, w, seed=3, offset=off)
         o = orc.verify_linear(w.target, w.draft, w.tokens, w.vocab, w.temperature, 3, off)
         assert g["status"] == 0 and np.all(o["err"] == 0)
-        compare_linear(g, o, w.k)
+        tally.add(compare_linear(g, o, w.k))
+    tally.check()
 
 
 @pytest.mark.parametrize("k", [1, 2, 7, 32])
 def test_draft_counts(sv, orc, k):
     w = wl.peaked_linear(seed=100 + k, batch=8, k=k, vocab=3000, temperature=1.0,
                          sigma=(0.2, 0.6))
+    tally = FlagTally()
     for off in range(4):
         g = run_linear_gpu(sv, w, seed=9, offset=off)
         o = orc.verify_linear(w.target, w.draft, w.tokens, w.vocab, w.temperature, 9, off)
-        compare_linear(g, o, w.k)
+        tally.add(compare_linear(g, o, w.k))
+    tally.check()
 
 
 def test_special_cases(sv, orc):
@@ -70,11 +77,12 @@ def test_special_cases(sv, orc):
     # q == p: every draft accepted, bonus from row k
     eq = wl.LinearWorkload("eq", w.target, np.ascontiguousarray(w.target[:, :4]), w.tokens, 64,
                            1.0, "f32")
+    tally = FlagTally()
     for off in range(10):
         g = run_linear_gpu(sv, eq, seed=1, offset=off)
         assert np.all(g["acc"] == 4)
         o = orc.verify_linear(eq.target, eq.draft, eq.tokens, 64, 1.0, 1, off)
-        compare_linear(g, o, 4)
+        tally.add(compare_linear(g, o, 4))
     # p_0(x_0) == 0: first draft always rejected, residual never returns x_0
     t = w.target.copy()
     for b in range(16):
@@ -84,8 +92,11 @@ def test_special_cases(sv, orc):
         g = run_linear_gpu(sv, z, seed=1, offset=off)
         assert np.all(g["acc"] == 0)
         assert np.all(g["out"][:, 0] != w.tokens[:, 0])
+        # log p_0(x_0) = -inf on both sides (checked by compare_linear)
+        assert np.all(np.isneginf(g["logp"][:, 0]))
         o = orc.verify_linear(z.target, z.draft, z.tokens, 64, 1.0, 1, off)
-        compare_linear(g, o, 4)
+        tally.add(compare_linear(g, o, 4))
+    tally.check()
 
 
 def test_input_errors_are_reported(sv, orc):
@@ -126,23 +137,40 @@ def test_host_side_argument_errors(sv):
         sv.spec_verify_linear(t2, d2, x, 16, 1.0)  # 72-byte rows are not 16-byte multiples
 
 
-@pytest.mark.parametrize("cfg", ["single", "batched"])
-def test_full_size_configs(sv, orc, cfg):
-    w = wl.config_single(seed=0) if cfg == "single" else wl.config_batched(seed=0)
-    offsets = range(24) if cfg == "single" else range(3)
-    tot = dict(trials=0, flagged_trials=0, flagged_mismatch=0)
+def _full_size(sv, orc, w, seed, offsets):
+    """GPU calls at every offset (inputs resident, outputs read once) against
+    the oracle's, spread over the host's cores; returns the tally and the
+    GPU's accepted lengths."""
+    dev = LinearOnDevice(sv, w)
+    gpu = dev.run_many(seed, offsets)
+    orcs = oracle_linear_many(orc, w, seed, offsets)
+    tally = FlagTally()
     lens = []
-    for off in offsets:
-        g = run_linear_gpu(sv, w, seed=123, offset=off)
-        o = orc.verify_linear(w.target, w.draft, w.tokens, w.vocab, w.temperature, 123, off)
+    for g, o in zip(gpu, orcs):
         assert g["status"] == 0
-        r = compare_linear(g, o, w.k)
-        for key in tot:
-            tot[key] += r[key]
+        tally.add(compare_linear(g, o, w.k))
         lens.extend(g["acc"].tolist())
-    print(cfg, tot, "mean accepted", np.mean(lens))
-    if cfg == "batched":
-        assert min(lens) == 0 or max(lens) == w.k or len(set(lens)) > 3
+    return tally, np.array(lens)
+
+
+def test_batched_config_100_offsets(sv, orc):
+    """B=64, k=8, V=128256 bf16, T=0.7 at 100 offsets: 6400 requests,
+    more than 2e4 decisions plus draws, so the 1e-4 flag budget is tested
+    against the expected rate of about 2e-5 per trial."""
+    w = wl.config_batched(seed=0)
+    tally, lens = _full_size(sv, orc, w, 123, range(100))
+    t = tally.check(min_trials=20_000)
+    print("batched", t, "mean accepted", lens.mean())
+    assert lens.min() == 0 and lens.max() == w.k  # residual and bonus draws both exercised
+
+
+def test_single_config_3000_steps(sv, orc):
+    """B=1, k=4, V=128256 bf16, T=1: 3000 seeded steps (offsets), more than
+    1e4 decisions plus draws."""
+    w = wl.config_single(seed=0)
+    tally, lens = _full_size(sv, orc, w, 123, range(3000))
+    t = tally.check(min_trials=10_000)
+    print("single", t, "mean accepted", lens.mean())
 
 
 def test_tiny_config_1e6_trials(sv, orc):
@@ -153,18 +181,16 @@ def test_tiny_config_1e6_trials(sv, orc):
     per_chunk, chunks = 250_000, 4
     outs = [[] for _ in range(base.batch)]
     accs = [[] for _ in range(base.batch)]
-    tot = dict(trials=0, flagged_trials=0, flagged_mismatch=0)
+    tally = FlagTally()
     for c in range(chunks):
         rep = wl.replicate_requests(base, per_chunk, draft_rng_seed=5000 + c)
         g = run_linear_gpu(sv, rep, seed=31, offset=c, dbg=False)
-        o = orc.verify_linear(rep.target, rep.draft, rep.tokens, rep.vocab, rep.temperature, 31, c)
-        r = compare_linear(g, o, rep.k, check_logp=False)
-        for key in tot:
-            tot[key] += r[key]
+        (o,) = oracle_linear_many(orc, rep, 31, [c])
+        tally.add(compare_linear(g, o, rep.k, check_logp=False))
         for b in range(base.batch):
             outs[b].append(g["out"][b * per_chunk:(b + 1) * per_chunk])
             accs[b].append(g["acc"][b * per_chunk:(b + 1) * per_chunk])
-    assert tot["flagged_trials"] <= 1e-4 * tot["trials"], tot
+    print("tiny 1e6", tally.check())
     for b in range(base.batch):
         out, acc = np.concatenate(outs[b]), np.concatenate(accs[b])
         for j in range(base.k + 1):
@@ -174,19 +200,45 @@ def test_tiny_config_1e6_trials(sv, orc):
             assert bad == 0 and pv > 1e-3, (b, j, pv)
 
 
+def test_brute_force_v8_k2_on_gpu(sv, orc):
+    """4e5 GPU trials at V=8, k=2 (fresh drafts each): the frequencies of
+    (accepted length, emitted tokens) match the exact joint enumerated over
+    every draft sequence, and every output equals the oracle's."""
+    V, k, T = 8, 2, 1.0
+    base = wl.tiny_linear(seed=21, batch=1, k=k, vocab=V)
+    p = softmax64(wl.as_f32(base.target, V), T)[0]
+    q = softmax64(wl.as_f32(base.draft, V), T)[0]
+    dist = brute_force_linear(p, q, k)
+    keys = sorted(dist)
+    index = {key: i for i, key in enumerate(keys)}
+    counts = np.zeros(len(keys))
+    tally = FlagTally()
+    unknown = 0
+    for c in range(4):
+        rep = wl.replicate_requests(base, 100_000, draft_rng_seed=7000 + c)
+        g = run_linear_gpu(sv, rep, seed=17, offset=c, dbg=False)
+        (o,) = oracle_linear_many(orc, rep, 17, [c])
+        tally.add(compare_linear(g, o, k, check_logp=False))
+        for row, n in zip(g["out"], g["acc"]):
+            key = (int(n),) + tuple(int(v) for v in row[:n + 1])
+            if key in index:
+                counts[index[key]] += 1
+            else:
+                unknown += 1
+    print("brute force v8 k2", tally.check(min_trials=400_000))
+    assert unknown == 0
+    pv, bad = chisquare_pvalue(counts, [dist[key] for key in keys])
+    assert bad == 0 and pv > 1e-3, pv
+
+
 def test_near_identical_rows_mark_many_entries(sv, orc):
     """Draft rows within ~1% of the target rows: residual draws whose p - q
     sign is undecided from fp32 for many entries (resolved exactly)."""
     w = wl.peaked_linear(seed=31, batch=32, k=32, vocab=20000, temperature=1.0,
                          sigma=(0.02, 0.02), dtype="f32")
-    residual = 0
-    for off in range(3):
-        g = run_linear_gpu(sv, w, seed=5, offset=off)
-        o = orc.verify_linear(w.target, w.draft, w.tokens, w.vocab, w.temperature, 5, off)
-        assert g["status"] == 0
-        compare_linear(g, o, w.k)
-        residual += int(np.sum(g["acc"] < w.k))
-    assert residual > 0
+    tally, lens = _full_size(sv, orc, w, 5, range(3))
+    tally.check()
+    assert int(np.sum(lens < w.k)) > 0
 
 
 def test_masked_vocabulary_is_never_drawn(sv, orc):
@@ -205,20 +257,42 @@ def test_masked_vocabulary_is_never_drawn(sv, orc):
     masked = np.zeros(V, bool)
     masked[15000:] = True
     masked[holes] = True
+    tally = FlagTally()
     for off in range(4):
         g = run_linear_gpu(sv, w, seed=9, offset=off)
         o = orc.verify_linear(w.target, w.draft, w.tokens, w.vocab, w.temperature, 9, off)
         assert g["status"] == 0
-        compare_linear(g, o, w.k)
+        tally.add(compare_linear(g, o, w.k))
         out = g["out"]
         assert not np.any(masked[out[out >= 0]])
+    tally.check()
 
 
 def test_more_requests_than_task_warps(sv, orc):
     """B = 700: the decide tasks outnumber the warps that take tasks first."""
     w = wl.peaked_linear(seed=51, batch=700, k=3, vocab=2000, temperature=1.0,
                          sigma=(0.5, 2.0), dtype="bf16")
-    g = run_linear_gpu(sv, w, seed=11, offset=0)
-    o = orc.verify_linear(w.target, w.draft, w.tokens, w.vocab, w.temperature, 11, 0)
+    tally, _ = _full_size(sv, orc, w, 11, range(1))
+    tally.check()
+
+
+def test_expired_waits_end_the_kernel_with_a_status(sv, orc):
+    """The diagnostic call stores no pass-1 partial, so every bounded wait
+    of the one-kernel path runs out: the kernel must return (no hang) with
+    SPEC_STATUS_TIMEOUT set and every output left at -1, and the next
+    normal call on the same workspace and context must be correct."""
+    w = wl.peaked_linear(seed=61, batch=8, k=4, vocab=20000, temperature=0.9,
+                         sigma=(0.5, 2.0), dtype="bf16")
+    tl, dl = to_device(w.target), to_device(w.draft)
+    x = to_device(w.tokens.astype(np.int32))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, acc = sv.spec_verify_debug_wait_expiry(tl, dl, x, w.vocab, w.temperature, 32, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & sv.STATUS_TIMEOUT
+    assert np.all(out.cpu().numpy() == -1) and np.all(acc.cpu().numpy() == -1)
+    tally = FlagTally()
+    g = run_linear_gpu(sv, w, seed=2, offset=0)
+    o = orc.verify_linear(w.target, w.draft, w.tokens, w.vocab, w.temperature, 2, 0)
     assert g["status"] == 0
-    compare_linear(g, o, w.k)
+    tally.add(compare_linear(g, o, w.k))
+    tally.check()
