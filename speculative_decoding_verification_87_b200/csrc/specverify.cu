@@ -1,7 +1,8 @@
 // specverify.cu -- C ABI of libspecverify.so (sm_100a) and its launches.
 //
-// spec_verify_linear: one cooperative launch of the persistent kernel
-// k_fused (sv_fused.cuh), which clears its own counters.
+// spec_verify_linear: one memset of the call's counters and pass-1
+// partials, then a cooperative launch of the persistent kernel k_fused
+// (sv_fused.cuh).
 // spec_verify_tree: the pass-1 kernel, the decide kernel and, where a token
 // is drawn, the pass-2 and finalize kernels (sv_verify.cuh), each a
 // programmatic dependent of the one before.
@@ -78,8 +79,8 @@ Layout layout(int B, int R, int V)
     const int64_t s2 = ceil_div(V, kSeg2);
     const int64_t w32 = s2 * (kSeg2 / 32);  // whole segments (16-byte aligned rows of the bitmap)
     size_t off = 0;
-    L.counters = off;  // p2cnt[B], decided[B], rowdone[B][R], p2claim, a_claim, p2ticket
-    off = align_up(off + sizeof(unsigned) * (static_cast<size_t>(B) * (R + 2) + 3));
+    L.counters = off;  // p2cnt[B], decided[B], p2claim, a_claim; rowpart follows directly
+    off = align_up(off + sizeof(unsigned) * (2 * static_cast<size_t>(B) + 2));
     L.rowpart = off;
     off = align_up(off + sizeof(float2) * static_cast<size_t>(B) * R * smax);
     L.req = off;
@@ -126,11 +127,8 @@ void fill_workspace(Params &p, void *ws, const Layout &L)
     auto *cnt = reinterpret_cast<unsigned *>(w + L.counters);
     p.p2cnt = cnt;
     p.decided = cnt + p.B;
-    p.rowdone = p.decided + p.B;
-    p.p2claim = p.rowdone + static_cast<int64_t>(p.B) * p.R;
+    p.p2claim = p.decided + p.B;
     p.a_claim = p.p2claim + 1;
-    p.p2ticket = p.a_claim + 1;
-    p.ncounters = static_cast<unsigned>(static_cast<int64_t>(p.B) * (p.R + 2) + 3);
     p.rowpart = reinterpret_cast<float2 *>(w + L.rowpart);
     p.req = reinterpret_cast<ReqInfo *>(w + L.req);
     p.p2part = reinterpret_cast<double4 *>(w + L.p2part);
@@ -275,12 +273,12 @@ int launch_verify(Params &p, const Layout &L, void *ws, int dtype_index, cudaStr
     return launch_dependent(k_finalize<Tag, MODE>, blocks3, dyn3, st, p);
 }
 
-// The one-kernel linear path: one cooperative launch (the kernel clears its
-// own counters before a grid-wide barrier), exactly one resident wave.  A
-// grid that cannot be resident at once fails to launch (SPEC_ECUDA).
+// The one-kernel linear path: clear the counters and partials, then one
+// cooperative launch, exactly one resident wave (a grid that cannot be
+// resident at once fails to launch: SPEC_ECUDA).
 int g_fused_blocks[64][2];
 template <class Tag>
-int launch_fused(Params &p, int dtype_index, cudaStream_t st)
+int launch_fused(Params &p, const Layout &L, void *ws, int dtype_index, cudaStream_t st)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SPEC_ECUDA;
@@ -294,6 +292,10 @@ int launch_fused(Params &p, int dtype_index, cudaStream_t st)
     // whole static rounds for about the first 88% of the pass-1 items
     const unsigned W = static_cast<unsigned>(per_sm * sms * kStreamers);
     p.nAs = static_cast<unsigned>((static_cast<uint64_t>(p.nA) * 88 / 100) / W * W);
+    // counters and pass-1 partials to all ones (kPartEmpty), one contiguous range
+    const size_t clear = L.rowpart - L.counters + sizeof(float2) * static_cast<size_t>(p.nA);
+    if (cudaMemsetAsync(static_cast<char *>(ws) + L.counters, 0xFF, clear, st) != cudaSuccess)
+        return SPEC_ECUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(per_sm * sms));
     cfg.blockDim = dim3(kThreads);
@@ -464,8 +466,6 @@ int setup_items(Params &p, int R, spec_dtype_t dtype, bool pass2)
     p.div_req = make_fastdiv(static_cast<uint32_t>(R) * static_cast<uint32_t>(p.S));
     p.div_s = make_fastdiv(static_cast<uint32_t>(p.S));
     p.div_s2 = make_fastdiv(static_cast<uint32_t>(p.S2));
-    const int chunk = dtype == SPEC_BF16 ? kP2ChunkBf16 : kP2ChunkF32;
-    p.div_cpr = make_fastdiv(static_cast<uint32_t>((p.S2 + chunk - 1) / chunk));
     return SPEC_OK;
 }
 
@@ -537,7 +537,8 @@ int linear_call(const void *target_logits, const void *draft_logits, spec_dtype_
     rc = setup_items(p, R, dtype, true);
     if (rc != SPEC_OK) return rc;
     fill_workspace(p, workspace, L);
-    return dtype == SPEC_BF16 ? launch_fused<Bf16>(p, 1, stream) : launch_fused<F32>(p, 0, stream);
+    return dtype == SPEC_BF16 ? launch_fused<Bf16>(p, L, workspace, 1, stream)
+                              : launch_fused<F32>(p, L, workspace, 0, stream);
 }
 
 }  // namespace

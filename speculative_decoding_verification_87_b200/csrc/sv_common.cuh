@@ -310,17 +310,11 @@ struct Params {
     unsigned *ambbits;       // [B][W32] undecided entries, one bit each
     double *p2w;             // [B][2][S2] finalize scratch (vocabularies too large for shared memory)
     double2 *p2lane;         // [B][S2][32] per-lane sums of pass 2 (decided part)
-    // one-kernel linear path: counters cleared to 0 (and rowpart set to all
-    // ones) by the kernel itself before its grid-wide barrier
+    // one-kernel linear path (set to all ones per call, with rowpart)
     unsigned *p2cnt;         // [B] pass-2 items completed per request
-    unsigned *decided;       // [B] 1 once the request's decision is published
-    unsigned *rowdone;       // [B][R] pass-1 items counted per row (relaxed; the partials
-                             //   themselves say whether they are complete)
-    unsigned *p2claim;       // decide tasks claimed
+    unsigned *p2claim;       // tasks claimed
     unsigned *a_claim;       // pass-1 chunks claimed past nAs
-    unsigned *p2ticket;      // pass-2 tickets claimed (request-major chunks of items)
-    unsigned ncounters;      // 32-bit words of the counters above (one contiguous range)
-    FastDiv div_cpr;         // by the pass-2 chunks per request
+    unsigned *decided;       // [B] 1 once the request's decision is published
     unsigned nAs;            // pass-1 items taken in static round robin
     unsigned poll_limit;     // polls before a wait gives up (SPEC_STATUS_TIMEOUT)
     int diag_no_partials;    // diagnostic only: pass 1 stores no partial, so every wait expires

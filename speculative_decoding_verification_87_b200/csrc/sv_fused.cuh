@@ -6,60 +6,40 @@
 // special-function, FMA and fp64 pipes and the memory system work at the
 // same time and no step waits for a whole grid.
 //
-//  * The kernel is launched cooperatively (every block resident at once,
-//    or the launch fails).  It first clears its own counters and sets every
-//    pass-1 partial to kPartEmpty (a bit pattern the reduction never
-//    stores) and every output to -1, then passes one grid-wide barrier;
-//    the streamers' first copies are already in flight across it.
 //  * Warps [0, kStreamers) of each block stream pass-1 items as k_pass1
 //    does (static round robin, no fences), the last part of them in
-//    chunks claimed from a counter, so faster SMs take more.  A partial
-//    that differs from kPartEmpty is complete.
-//  * Each stored partial is also counted on its row (rowdone, a relaxed
-//    atomic without a fence: the count may become visible before the
-//    partial, so a reader checks the partials themselves).
+//    chunks claimed from a counter, so faster SMs take more.  Before the
+//    kernel every partial holds kPartEmpty, a bit pattern the reduction
+//    never stores, so a partial that differs from it is complete.
 //  * The other warps, and every streamer once its pass-1 items are done,
-//    first take the B decide tasks from a counter (each starts as early as
-//    possible).  A decide task polls its request's R row counts (one word
-//    per lane, bounded) until every row is counted complete, reads the
-//    partials (re-reading any still empty), merges each row across the warp,
-//    decides ("Speculative decoding explained", section "Draft and
-//    verification loop") and publishes decided[b].
-//  * Then they take pass-2 tickets from one counter, in request order: a
-//    ticket is a chunk of a request's items (segments of the row or row pair
-//    of its final draw).  A worker keeps two tickets in flight: the next
-//    one's rows are copied into shared memory while the current one is
-//    reduced in fp64, published, and counted with one fence and one atomic;
-//    the warp that completes a request's last item draws its token.  An
-//    expired wait sets SPEC_STATUS_TIMEOUT and the warp leaves.
+//    take tasks from a shared counter: first the B decide tasks (each starts
+//    as early as possible), then the B * S2 pass-2 items in request order.
+//    The decide task polls the
+//    request's partials (uncached loads, bounded) until none is empty,
+//    merges its rows, decides ("Speculative decoding explained", section
+//    "Draft and verification loop") and publishes decided[b].  A pass-2
+//    item waits (bounded) for decided[b], is reduced, and arrives on the
+//    request's counter; the warp that completes the last draws the token.
+//    An expired wait sets SPEC_STATUS_TIMEOUT and the warp leaves.
 //
 // Progress: streamers wait on nothing; a decide task waits only on
-// streamers; a pass-2 worker waits only on decide tasks, which are claimed
-// (and so running) before any warp takes a ticket.
+// streamers; an item waits only on its request's decide task, which was
+// claimed earlier by a running warp.  The grid is one resident wave, and
+// the launch is cooperative, so a grid that cannot be resident at once
+// fails to launch instead of leaving a wait to expire.
 #pragma once
-
-#include <cooperative_groups.h>
 
 #include "sv_verify.cuh"
 
 namespace sv {
 
 constexpr int kStreamers = 6;        // pass-1 warps per block
-constexpr int kFusedRing = 3;        // ring slots of a streamer (kFusedRing - 1 items in flight)
-constexpr int kRegion = 640;         // uint4 (10 KB): a task warp's scratch
-// a streamer's region holds its ring, and later (when it takes tasks) the
-// task scratch
-constexpr int kRegionS = kFusedRing * 256 > kRegion ? kFusedRing * 256 : kRegion;
-static_assert(256 == 32 * 8, "a ring slot is one pass-1 item (256 uint4)");
-constexpr size_t kFusedSmem = sizeof(uint4) * (kRegionS * kStreamers + kRegion * (kWarps - kStreamers));
-constexpr unsigned kWaitPolls = 1u << 20;  // ~1 s of polling at <= 1 us per poll
-// pass-2 items per ticket: two 2 KB segments (bf16), one 4 KB segment (fp32)
-constexpr int kP2ChunkBf16 = 2;
-constexpr int kP2ChunkF32 = 1;
-template <class Tag>
-constexpr int p2_chunk() { return Tag::kVec == 8 ? kP2ChunkBf16 : kP2ChunkF32; }
-// An empty partial: all bits set.  A stored partial's max is never this
-// NaN: NaN maxima are canonical.
+constexpr int kRegion = 3 * 256;     // uint4 per warp (12 KB): pass-1 ring, later task scratch
+static_assert(kRing1 * 32 * 8 <= kRegion, "the pass-1 ring fits a warp region");
+constexpr size_t kFusedSmem = sizeof(uint4) * kRegion * kWarps;
+constexpr unsigned kWaitPolls = 1u << 20;  // ~1 s of polling at <= 1 us per poll (Params::poll_limit)
+// An empty partial / counter word: all bits set (one memset per call).  A
+// stored partial's max is never this NaN: NaN maxima are canonical.
 constexpr unsigned kPartEmpty = 0xFFFFFFFFu;
 
 // Polling reads: fetched again on every call (never from a stale L1 line)
@@ -71,10 +51,10 @@ __device__ __forceinline__ unsigned long long ld_poll64(const void *p)
 }
 __device__ __forceinline__ unsigned ld_poll32(const unsigned *p) { return __ldcv(p); }
 
-__device__ __forceinline__ void backoff(unsigned &ns, unsigned cap = 1024)
+__device__ __forceinline__ void backoff(unsigned &ns)
 {
     __nanosleep(ns);
-    ns = ns < cap ? 2 * ns : cap;
+    ns = ns < 1024 ? 2 * ns : 1024;
 }
 
 // Merge one row's S partials (one lane), in two passes so that the terms
@@ -104,31 +84,14 @@ __device__ __forceinline__ void merge_row_lane(const Params &p, Load part, float
     S = nan ? __longlong_as_double(0x7FF8000000000000ll) : s;
 }
 
-// Before the grid-wide barrier: counters to 0, pass-1 partials to
-// kPartEmpty, outputs to -1 (what a request keeps if a wait expires).
-__device__ __forceinline__ void fused_init(const Params &p)
-{
-    const unsigned tid = blockIdx.x * blockDim.x + threadIdx.x;
-    const unsigned nth = gridDim.x * blockDim.x;
-    for (unsigned i = tid; i < p.ncounters; i += nth) p.p2cnt[i] = 0u;
-    uint2 *part = reinterpret_cast<uint2 *>(p.rowpart);
-    for (unsigned i = tid; i < p.nA; i += nth) part[i] = make_uint2(kPartEmpty, kPartEmpty);
-    const unsigned nout = static_cast<unsigned>(p.B) * static_cast<unsigned>(p.k + 1);
-    for (unsigned i = tid; i < nout; i += nth) p.out[i] = -1;
-    for (unsigned i = tid; i < static_cast<unsigned>(p.B); i += nth) p.acc[i] = -1;
-}
-
 // The streamer of the fused kernel.  Items [0, nAs) are taken in static
 // round robin (as in pass1_stream); the rest, in chunks of kDynChunk
 // consecutive items from a shared counter, claimed one chunk ahead just
 // before the warp needs it, so the SMs that run faster take more of the
 // tail.  Lane q holds the item id of slot q (kNoItem: the sequence ended).
-// The ring is first filled with static items only, before the grid-wide
-// barrier (no counter may be touched before it); then the barrier.
 constexpr unsigned kDynChunk = 4;
 template <class Tag>
-__device__ __forceinline__ void fused_stream(const Params &p, uint4 *ring, unsigned w, unsigned W,
-                                             bool streamer)
+__device__ __forceinline__ void fused_stream(const Params &p, uint4 *ring, unsigned w, unsigned W)
 {
     constexpr int kSlot = Pass1Shape<Tag>::kSlot;
     const int lane = threadIdx.x & 31;
@@ -137,7 +100,7 @@ __device__ __forceinline__ void fused_stream(const Params &p, uint4 *ring, unsig
     unsigned claim = 0;               // lane 0: the chunk claimed ahead
     bool claimed = false, done = false;
     auto claim_ahead = [&]() {
-        if (lane == 0) claim = atomicAdd(p.a_claim, 1u);
+        if (lane == 0) claim = atomicAdd(p.a_claim, 1u) + 1u;  // the counter starts at all ones
         claimed = true;
     };
     auto next_item = [&]() -> unsigned {
@@ -169,38 +132,26 @@ __device__ __forceinline__ void fused_stream(const Params &p, uint4 *ring, unsig
         if (lane == q) meta = it;
         commit_copies();
     };
-    // prologue: static items only (a static item whose successor would be
-    // claimed stops the prologue before that claim)
-    int filled = 0;
-    if (streamer) {
 #pragma unroll 1
-        for (; filled < kFusedRing && st < p.nAs && st + W < p.nAs; ++filled) refill(filled);
-    }
-    cooperative_groups::this_grid().sync();
-    if (!streamer) return;
-#pragma unroll 1
-    for (; filled < kFusedRing; ++filled) refill(filled);
+    for (int q = 0; q < kRing1; ++q) refill(q);
     int q = 0;
 #pragma unroll 1
     for (;;) {
-        wait_copies<kFusedRing - 1>();
+        wait_copies<kRing1 - 1>();
         const unsigned it = __shfl_sync(kFull, meta, q);
         if (it == kNoItem) break;
         const int s = static_cast<int>(it - fdiv(it, p.div_s) * static_cast<unsigned>(p.S));
         reduce_item1<Tag, kLinear>(p, it, s, ring + q * kSlot);
-        if (lane == 0) atomicAdd(p.rowdone + fdiv(it, p.div_s), 1u);  // no fence: a hint only
         refill(q);
-        q = (q + 1 == kFusedRing) ? 0 : q + 1;
+        q = (q + 1 == kRing1) ? 0 : q + 1;
     }
     wait_copies<0>();
 }
 
-// The decide task of request b: wait until every row of the request is
-// counted complete, then until every partial is stored (the counts carry no
-// fence, so a partial still empty is read again), merge each row across the
-// warp, decide, publish.  scr: the warp's region (the partials are staged
-// there when they fit, else read again through L2).  False when a wait
-// expired.
+// The decide task of request b: wait until all its pass-1 partials are
+// stored, merge its rows (a lane per row), decide, publish.  scr: the
+// warp's region; R*S partials are staged there when they fit, else
+// re-read through L2.  False when the wait expired.
 template <class Tag>
 __device__ __forceinline__ bool decide_task(const Params &p, int b, uint4 *scr)
 {
@@ -208,55 +159,46 @@ __device__ __forceinline__ bool decide_task(const Params &p, int b, uint4 *scr)
     const DraftProbe pr = probe_drafts<Tag>(p, b);  // inputs: read while pass 1 runs
     const int n = p.R * p.S;
     const float2 *part = p.rowpart + static_cast<int64_t>(b) * n;
-    const unsigned *cnt = p.rowdone + static_cast<int64_t>(b) * p.R;
     float2 *stg = reinterpret_cast<float2 *>(scr);
     const bool staged = static_cast<size_t>(n) * sizeof(float2) + sizeof(double) * 2 * 65 <=
                         sizeof(uint4) * kRegion;
     bool done = false;
-    unsigned it = 0, ns = 64;
-    for (; it < p.poll_limit; ++it) {
+    unsigned ns = 64;
+    for (unsigned it = 0; it < p.poll_limit; ++it) {
         bool all = true;
-        for (int r = lane; r < p.R; r += 32) all &= ld_poll32(cnt + r) >= static_cast<unsigned>(p.S);
+        for (int i = lane; i < n; i += 32) {
+            const unsigned long long v = ld_poll64(part + i);
+            all &= static_cast<unsigned>(v) != kPartEmpty;
+            if (staged) stg[i] = make_float2(__uint_as_float(static_cast<unsigned>(v)),
+                                             __uint_as_float(static_cast<unsigned>(v >> 32)));
+        }
         if (__all_sync(kFull, all)) {
             done = true;
             break;
         }
-        backoff(ns, 1024);
+        backoff(ns);
     }
-    // every partial counted: read them all, again only those still empty
-    bool have = false;
-    if (done) {
-        bool first = true;  // the first round reads every partial
-        for (; it < p.poll_limit; ++it) {
-            bool all = true;
-            for (int i = lane; i < n; i += 32) {
-                if (staged && !first && __float_as_uint(stg[i].x) != kPartEmpty) continue;
-                const unsigned long long v = ld_poll64(part + i);
-                all &= static_cast<unsigned>(v) != kPartEmpty;
-                if (staged)
-                    stg[i] = make_float2(__uint_as_float(static_cast<unsigned>(v)),
-                                         __uint_as_float(static_cast<unsigned>(v >> 32)));
-            }
-            first = false;
-            if (__all_sync(kFull, all)) break;
-            __nanosleep(64);
+    if (!done) {
+        // the request is given up: its outputs read -1
+        for (int j = lane; j <= p.k; j += 32) p.out[static_cast<int64_t>(b) * (p.k + 1) + j] = -1;
+        if (lane == 0) {
+            p.acc[b] = -1;
+            report(p.status, kStTimeout);
         }
-        have = it < p.poll_limit;
-    }
-    if (!have) {
-        if (lane == 0) report(p.status, kStTimeout);
         return false;
     }
     __syncwarp();
-    // a lane per row (its partials from shared memory; no shuffles, so the
-    // chain stays short on a warp that shares its scheduler with streamers)
     double *ds = reinterpret_cast<double *>(scr + kRegion) - 65;
     float *dm = reinterpret_cast<float *>(ds) - 65;
     for (int r = lane; r < p.R; r += 32) {
         float M;
         double S;
-        if (staged) merge_row_lane(p, [&](int j) { return stg[r * p.S + j]; }, M, S);
-        else merge_row_lane(p, [&](int j) { return __ldcg(part + r * p.S + j); }, M, S);
+        if (staged) {
+            merge_row_lane(p, [&](int j) { return stg[r * p.S + j]; }, M, S);
+        } else {
+            // not staged: the values are final now; read them through L2
+            merge_row_lane(p, [&](int j) { return __ldcg(part + r * p.S + j); }, M, S);
+        }
         dm[r] = M;
         ds[r] = S;
     }
@@ -286,7 +228,7 @@ __device__ __forceinline__ bool wait_decided(const Params &p, int b)
                 ok = 1;
                 break;
             }
-            backoff(ns, 512);
+            backoff(ns);
         }
         if (ok) __threadfence();
         else report(p.status, kStTimeout);
@@ -294,125 +236,60 @@ __device__ __forceinline__ bool wait_decided(const Params &p, int b)
     return __shfl_sync(kFull, ok, 0) != 0;
 }
 
-// A pass-2 ticket: items [c0, c1) of request b.
-struct Ticket {
-    int b, c0, c1;
-    ItemInfo it;
-    bool valid;  // a ticket of the call (past the last: the worker is done)
-    bool work;   // the request draws a token (else its tickets are empty)
-};
-
-// Take the next ticket, wait until its request is decided and read its
-// record (unless it is the request of `prev`), and start the copies of its
-// rows into buf (one commit group, empty when there is nothing to copy).
-// False when a wait expired.
-template <class Tag>
-__device__ __forceinline__ bool take_ticket(const Params &p, Ticket &t, const Ticket &prev, uint4 *buf,
-                                            unsigned &ahead)
-{
-    constexpr int kCh = p2_chunk<Tag>();
-    const int lane = threadIdx.x & 31;
-    // the ticket number was claimed one ticket ahead (lane 0), so the
-    // atomic's round trip overlaps the work in between
-    unsigned x = __shfl_sync(kFull, ahead, 0);
-    if (lane == 0) ahead = atomicAdd(p.p2ticket, 1u);
-    const unsigned cpr = p.div_cpr.d;
-    t.valid = x < static_cast<unsigned>(p.B) * cpr;
-    t.work = false;
-    if (t.valid) {
-        t.b = static_cast<int>(fdiv(x, p.div_cpr));
-        const int c = static_cast<int>(x - static_cast<unsigned>(t.b) * cpr);
-        t.c0 = c * kCh;
-        t.c1 = min(t.c0 + kCh, p.S2);
-        if (prev.valid && prev.b == t.b) {
-            t.it = prev.it;
-        } else {
-            if (!wait_decided(p, t.b)) {
-                commit_copies();
-                return false;
-            }
-            t.it = load_item_info(p, t.b);
-        }
-        t.work = t.it.mode == kModeResidual || t.it.mode == kModeTargetRow;
-        if (t.work)
-            for (int s2 = t.c0; s2 < t.c1; ++s2) {
-                uint4 *sb = buf + (s2 - t.c0) * StageShape<Tag>::kPerBuf;
-                if (t.it.mode == kModeResidual) stage_item<Tag, true>(p, t.it, s2, sb);
-                else stage_item<Tag, false>(p, t.it, s2, sb);
-            }
-    }
-    commit_copies();
-    return true;
-}
-
-// Reduce and publish a staged ticket, count its items with one fence and
-// one atomic; true when it completed its request (the caller then draws).
-template <class Tag>
-__device__ __forceinline__ bool finish_ticket(const Params &p, const Ticket &t, const uint4 *buf,
-                                              const double *tab)
-{
-    const int lane = threadIdx.x & 31;
-    const bool residual = t.it.mode == kModeResidual;
-    for (int s2 = t.c0; s2 < t.c1; ++s2) {
-        const uint4 *sb = buf + (s2 - t.c0) * StageShape<Tag>::kPerBuf;
-        if (residual) p2_item<Tag, true>(p, t.b, s2, t.it, sb, tab);
-        else p2_item<Tag, false>(p, t.b, s2, t.it, sb, tab);
-    }
-    __threadfence();  // every lane's stores of the ticket precede its count
-    __syncwarp();
-    unsigned o = 0;
-    const unsigned nc = static_cast<unsigned>(t.c1 - t.c0);
-    if (lane == 0) {
-        o = atomicAdd(&p.p2cnt[t.b], nc) + nc;
-        if (o == static_cast<unsigned>(p.S2)) __threadfence();
-    }
-    return __shfl_sync(kFull, o == static_cast<unsigned>(p.S2) ? 1 : 0, 0) != 0;
-}
-
-// The task worker: decide tasks first (claimed from a counter), then pass-2
-// tickets, two in flight.
+// The task worker: tasks in request order from the shared counter (which
+// starts at kPartEmpty, so a claim returns the task id minus one).
 template <class Tag>
 __device__ __forceinline__ void fused_tasks(const Params &p, uint4 *region, const double *tab)
 {
     const int lane = threadIdx.x & 31;
-    constexpr int kBuf = p2_chunk<Tag>() * StageShape<Tag>::kPerBuf;  // uint4 per ticket
-    static_assert(2 * kBuf <= kRegion, "two tickets' staging fit a warp region");
-    double *W_sh = reinterpret_cast<double *>(region + 2 * kBuf);
+    // one staging buffer (an item is staged and reduced in turn), then the
+    // finalize scratch
+    static_assert(StageShape<Tag>::kPerBuf <= kRegion, "a staging buffer fits a warp region");
+    uint4 *stage = region;
+    double *W_sh = reinterpret_cast<double *>(region + StageShape<Tag>::kPerBuf);
     const bool w_shared = 2 * static_cast<size_t>(p.S2) * sizeof(double) <=
-                          sizeof(uint4) * static_cast<size_t>(kRegion - 2 * kBuf);
-    const unsigned B = static_cast<unsigned>(p.B);
-    // decide tasks: a task is claimed only by a free warp, which starts it
-    // at once, so no pass-2 worker waits on a decide that nobody runs
-#pragma unroll 1
-    for (;;) {
+                          sizeof(uint4) * static_cast<size_t>(kRegion - StageShape<Tag>::kPerBuf);
+    // tasks [0, B): the decide steps; then B * S2 items in request order
+    const unsigned ntask = static_cast<unsigned>(p.B) * (static_cast<unsigned>(p.S2) + 1u);
+    // a task is claimed only by a free warp: a claimed decide task starts at
+    // once, so no item waits on a decide that waits on that item's warp
+    auto claim = [&]() {
         unsigned t = 0;
-        if (lane == 0) t = atomicAdd(p.p2claim, 1u);
-        t = __shfl_sync(kFull, t, 0);
-        if (t >= B) break;
-        if (!decide_task<Tag>(p, static_cast<int>(t), region)) return;
-    }
-    // pass 2: tickets in request order, the next one copied while the
-    // current one is reduced
-    Ticket none;
-    none.valid = false;
-    Ticket cur, nxt;
-    int q = 0;
-    unsigned ahead = 0;
-    if (lane == 0) ahead = atomicAdd(p.p2ticket, 1u);
-    if (!take_ticket<Tag>(p, cur, none, region, ahead)) return;
+        if (lane == 0) t = atomicAdd(p.p2claim, 1u) + 1u;
+        return __shfl_sync(kFull, t, 0);
+    };
+    unsigned cur = claim();
 #pragma unroll 1
-    while (cur.valid) {
-        if (!take_ticket<Tag>(p, nxt, cur, region + (q ^ 1) * kBuf, ahead)) {
-            wait_copies<0>();
-            return;
+    while (cur < ntask) {
+        if (cur < static_cast<unsigned>(p.B)) {
+            if (!decide_task<Tag>(p, static_cast<int>(cur), region)) break;
+        } else {
+            const unsigned item = cur - static_cast<unsigned>(p.B);
+            const int b = static_cast<int>(fdiv(item, p.div_s2));
+            const int s2 = static_cast<int>(item - static_cast<unsigned>(b) * static_cast<unsigned>(p.S2));
+            if (!wait_decided(p, b)) break;
+            const ItemInfo it = load_item_info(p, b);
+            if (it.mode == kModeResidual || it.mode == kModeTargetRow) {
+                if (it.mode == kModeResidual) stage_item<Tag, true>(p, it, s2, stage);
+                else stage_item<Tag, false>(p, it, s2, stage);
+                commit_copies();
+                wait_copies<0>();
+                if (it.mode == kModeResidual) p2_item<Tag, true>(p, b, s2, it, stage, tab);
+                else p2_item<Tag, false>(p, b, s2, it, stage, tab);
+                __threadfence();  // every lane's stores of the item precede its arrival
+                __syncwarp();
+                unsigned o = 0;
+                if (lane == 0) {
+                    o = atomicAdd(&p.p2cnt[b], 1u) + 1u;  // the counter starts at kPartEmpty
+                    if (o == static_cast<unsigned>(p.S2) - 1u) __threadfence();
+                }
+                if (__shfl_sync(kFull, o == static_cast<unsigned>(p.S2) - 1u ? 1 : 0, 0)) {
+                    double *W = w_shared ? W_sh : p.p2w + 2 * static_cast<int64_t>(b) * p.S2;
+                    finalize<Tag>(p, b, tab, W, W + p.S2);
+                }
+            }
         }
-        wait_copies<1>();  // the current ticket's copies have landed
-        if (cur.work && finish_ticket<Tag>(p, cur, region + q * kBuf, tab)) {
-            double *W = w_shared ? W_sh : p.p2w + 2 * static_cast<int64_t>(cur.b) * p.S2;
-            finalize<Tag>(p, cur.b, tab, W, W + p.S2);
-        }
-        cur = nxt;
-        q ^= 1;
+        cur = claim();
     }
     wait_copies<0>();
 }
@@ -423,13 +300,11 @@ __global__ void __launch_bounds__(kThreads, 2) k_fused(const __grid_constant__ P
     extern __shared__ uint4 fdyn[];
     __shared__ double tab[kExp2Tab];
     for (int j = threadIdx.x; j < kExp2Tab; j += kThreads) tab[j] = p.exp2tab[j];
-    fused_init(p);
     __syncthreads();
     const int warp = threadIdx.x >> 5;
-    uint4 *region = warp < kStreamers ? fdyn + warp * kRegionS
-                                      : fdyn + kStreamers * kRegionS + (warp - kStreamers) * kRegion;
-    // every warp reaches the grid-wide barrier inside fused_stream
-    fused_stream<Tag>(p, region, blockIdx.x * kStreamers + warp, gridDim.x * kStreamers, warp < kStreamers);
+    uint4 *region = fdyn + warp * kRegion;
+    if (warp < kStreamers)
+        fused_stream<Tag>(p, region, blockIdx.x * kStreamers + warp, gridDim.x * kStreamers);
     fused_tasks<Tag>(p, region, tab);
 }
 
