@@ -41,7 +41,8 @@ METRIC = "verify rows/s and achieved HBM GB/s (B=64, k=8, V=128256 bf16, 1 B200)
 KERNEL_OF = {
     "batched": "k_fused (one launch per call, after a 0.55 MB memset)",
     "single": "k_fused (one launch per call, after a memset)",
-    "greedy": "k_greedy_cluster (one launch per call)",
+    "greedy": "k_pass1 + k_greedy_decide (programmatic dependent; workspace form)",
+    "greedy-cluster": "k_greedy_cluster (one launch per call; the workspace-free form)",
     "tree": "k_pass1 + k_decide (programmatic dependents)",
     "tree-stochastic": "k_pass1 + k_decide + k_pass2 + k_finalize (programmatic dependents)",
     "tree-exact": "k_pass1 + k_tree_exact (programmatic dependent)",
@@ -120,7 +121,7 @@ def make_workload(name, seed):
         return wl.config_batched(seed=seed)
     if name == "single":
         return wl.config_single(seed=seed)
-    if name in ("greedy", "greedy-walk"):
+    if name in ("greedy", "greedy-cluster", "greedy-walk"):
         return wl.config_greedy(seed=seed)
     if name in TREES:
         return wl.config_tree(seed=seed)
@@ -164,12 +165,13 @@ def workload_facts(name, w):
         io = B * k * 4 + B * (k + 1) * 4 + B * 4
         cfg = dict(workload=f"linear stochastic verify B={B} k={k} V={V} {w.dtype} T={w.temperature}",
                    batch=B, k=k, vocab=V, temperature=w.temperature)
-    elif name == "greedy":
+    elif name in ("greedy", "greedy-cluster"):
         B, k, V = w.batch, w.k, w.vocab
         rows = B * (k + 1)
         logits = B * (k + 1) * V * esz
         io = B * k * 4 + B * (k + 1) * 4 + B * 4
-        cfg = dict(workload=f"linear greedy verify B={B} k={k} V={V} {w.dtype}", batch=B, k=k,
+        form = " (workspace-free form)" if name == "greedy-cluster" else ""
+        cfg = dict(workload=f"linear greedy verify{form} B={B} k={k} V={V} {w.dtype}", batch=B, k=k,
                    vocab=V)
     else:
         B, N, V = w.batch, w.num_nodes, w.vocab
@@ -348,8 +350,9 @@ class Runner:
         else:
             self.tokens = dev(w.tokens.astype(np.int32))
             self.out = torch.empty((w.batch, w.k + 1), dtype=torch.int32, device=device)
-            # greedy: a cluster kernel; linear stochastic: k_fused
-            self.kernels_per_call = 1
+            # linear stochastic: k_fused; greedy: k_pass1 + k_greedy_decide, or
+            # the cluster kernel alone
+            self.kernels_per_call = 2 if name == "greedy" else 1
         self.acc = torch.empty((w.batch,), dtype=torch.int32, device=device)
 
     def clone(self):
@@ -373,9 +376,9 @@ class Runner:
         if self.name in ("batched", "single"):
             b.spec_verify_linear(target, draft, tokens, w.vocab, w.temperature, 1234, offset,
                                  out_tokens=self.out, accepted_len=self.acc)
-        elif self.name == "greedy":
+        elif self.name in ("greedy", "greedy-cluster"):
             b.spec_verify_greedy(target, tokens, w.vocab, out_tokens=self.out,
-                                 accepted_len=self.acc)
+                                 accepted_len=self.acc, workspace_free=self.name == "greedy-cluster")
         elif self.name == "greedy-walk":
             b.spec_verify_greedy_walk(target, tokens, w.vocab, out_tokens=self.out,
                                       accepted_len=self.acc)
@@ -571,7 +574,7 @@ def oracle_call(name, s, offset):
     if name in ("batched", "single"):
         oracle.verify_linear(s.target, s.draft, s.tokens, s.vocab, s.temperature, 1234, offset)
         return s.target.shape[0] * s.target.shape[1]
-    if name in ("greedy", "greedy-walk"):
+    if name in ("greedy", "greedy-cluster", "greedy-walk"):
         oracle.verify_greedy(s.target, s.tokens, s.vocab)
         return s.target.shape[0] * s.target.shape[1]
     if name == "tree-exact":
@@ -663,7 +666,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="batched",
-                    choices=["batched", "single", "greedy", "tree", "tree-stochastic", "tree-exact",
+                    choices=["batched", "single", "greedy", "greedy-cluster", "tree", "tree-stochastic",
+                             "tree-exact",
                              "greedy-walk", "tree-walk"])
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--l2", choices=["cold", "warm"], default="cold",

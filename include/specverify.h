@@ -182,13 +182,19 @@ SPECVERIFY_API int spec_verify_linear_noalloc(const void *target_logits, const v
  * lowest index; n = first j < k with draft_tokens[b][j] != g_j, else k.
  * Outputs: out_tokens [B][k+1] = x_0..x_{n-1}, g_n, then -1; accepted_len [B] = n.
  * Draft logits are not read and the temperature does not apply.
- * Needs no workspace: the argmax of a request is merged across a thread-block
- * cluster in distributed shared memory.
+ * workspace: NULL, or at least spec_verify_workspace_size(B, k+1, V) bytes,
+ *   256-byte aligned (else SPEC_EWORKSPACE; workspace_bytes is ignored when
+ *   workspace is NULL).  Both forms give identical outputs.  With a
+ *   workspace the rows are streamed in fixed-size items whose partial
+ *   (max, argmax) records the workspace holds, then merged per row: the
+ *   faster form.  Without one, a thread-block cluster merges each request's
+ *   argmax in distributed shared memory, for callers that cannot provide
+ *   device memory.  A workspace must not be shared by calls that may overlap.
  */
 SPECVERIFY_API int spec_verify_greedy(const void *target_logits, spec_dtype_t dtype, int64_t row_stride,
                        const int32_t *draft_tokens, int batch, int k, int vocab,
                        int32_t *out_tokens, int32_t *accepted_len, int32_t *status,
-                       cudaStream_t stream);
+                       void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * Tree verification ("Accelerating Sonar through speculation", section

@@ -60,7 +60,7 @@ def load_library(path: str = LIB_PATH):
         L.spec_verify_linear.argtypes = [_P, _P, _I, _I64, _P, _I, _I, _I, _F, _U64, _U32, _P, _P,
                                          _P, _P, _P, _P, _SZ, _P]
         L.spec_verify_linear.restype = _I
-        L.spec_verify_greedy.argtypes = [_P, _I, _I64, _P, _I, _I, _I, _P, _P, _P, _P]
+        L.spec_verify_greedy.argtypes = [_P, _I, _I64, _P, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]
         L.spec_verify_greedy.restype = _I
         L.spec_verify_tree.argtypes = [_P, _P, _I, _I64, _P, _P, _I, _I, _I, _I, _I, _F, _U64,
                                        _U32, _P, _P, _P, _P, _P, _SZ, _P]
@@ -191,8 +191,10 @@ def spec_verify_linear(target_logits, draft_logits, draft_tokens, vocab, tempera
 
 
 def spec_verify_greedy(target_logits, draft_tokens, vocab, out_tokens=None, accepted_len=None,
-                       status=None, stream=None):
-    """target_logits [B][k+1][stride], draft_tokens [B][k] int32."""
+                       status=None, workspace_buf=None, stream=None, workspace_free=False):
+    """target_logits [B][k+1][stride], draft_tokens [B][k] int32.  By default
+    the streamed form runs in a cached workspace (or workspace_buf);
+    workspace_free=True runs the cluster form, which needs none."""
     _need_cuda("target_logits", target_logits)
     B, R, stride = target_logits.shape
     k = R - 1
@@ -206,9 +208,15 @@ def spec_verify_greedy(target_logits, draft_tokens, vocab, out_tokens=None, acce
     _need_cuda("accepted_len", accepted_len, torch.int32, (B,))
     if status is not None:
         _need_cuda("status", status, torch.int32)
+    if workspace_free:
+        workspace_buf = None
+    elif workspace_buf is None and B > 0:
+        workspace_buf = workspace(B, k + 1, vocab, dev)
+    ws_bytes = 0 if workspace_buf is None else workspace_buf.numel()
     rc = load_library().spec_verify_greedy(
         _ptr(target_logits), _dtype_code(target_logits), stride, _ptr(draft_tokens), B, k, vocab,
-        _ptr(out_tokens), _ptr(accepted_len), _ptr(status), _stream(stream))
+        _ptr(out_tokens), _ptr(accepted_len), _ptr(status), _ptr(workspace_buf), ws_bytes,
+        _stream(stream))
     _check(rc, "spec_verify_greedy")
     return out_tokens, accepted_len
 

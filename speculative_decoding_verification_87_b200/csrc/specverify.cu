@@ -6,8 +6,9 @@
 // spec_verify_tree: the pass-1 kernel, the decide kernel and, where a token
 // is drawn, the pass-2 and finalize kernels (sv_verify.cuh), each a
 // programmatic dependent of the one before.
-// spec_verify_greedy: one launch of the cluster kernel (sv_greedy.cuh); no
-// workspace.
+// spec_verify_greedy: with a workspace, k_pass1 (greedy tree mode over the
+// target rows) and k_greedy_decide; without one, one launch of the cluster
+// kernel k_greedy_cluster (sv_greedy.cuh).
 // Everything is enqueued on the caller's stream; no host synchronisation.
 #include <algorithm>
 #include <climits>
@@ -219,6 +220,16 @@ int launch_dependent(Kernel kernel, int64_t blocks, size_t dyn, cudaStream_t st,
     return cudaLaunchKernelEx(&cfg, kernel, p) == cudaSuccess ? SPEC_OK : SPEC_ECUDA;
 }
 
+// Pass 1's static share (whole rounds of the grid's warps for about 88% of
+// the items; the rest is claimed in chunks) and its claim counter, set to
+// all ones on the stream before the launch.
+int prep_pass1(Params &p, int64_t blocks, cudaStream_t st)
+{
+    const uint64_t W = static_cast<uint64_t>(blocks) * kWarps;
+    p.nAs = static_cast<unsigned>((static_cast<uint64_t>(p.nA) * 88 / 100) / W * W);
+    return cudaMemsetAsync(p.a_claim, 0xFF, sizeof(unsigned), st) == cudaSuccess ? SPEC_OK : SPEC_ECUDA;
+}
+
 // Launch pass 1, then the decide step and, where a token is drawn, pass 2
 // and the finalize step, each a programmatic dependent of the one before.
 // Pass grids are at most one resident wave.
@@ -258,6 +269,7 @@ int launch_verify(Params &p, const Layout &L, void *ws, int dtype_index, cudaStr
     if (per_sm1 < 1 || per_sm2 < 1 || sms < 1) return SPEC_ECUDA;
     const int64_t blocks1 =
         std::max<int64_t>(1, std::min<int64_t>(static_cast<int64_t>(per_sm1) * sms, ceil_div(p.nA, kWarps)));
+    if (prep_pass1(p, blocks1, st) != SPEC_OK) return SPEC_ECUDA;
     k_pass1<Tag, MODE, kMin1><<<static_cast<unsigned>(blocks1), kThreads, kRingBytes, st>>>(p);
     if (cudaGetLastError() != cudaSuccess) return SPEC_ECUDA;
     const int64_t blocksd = std::max<int64_t>(1, std::min<int64_t>(static_cast<int64_t>(2) * sms, p.B));
@@ -350,6 +362,7 @@ int launch_exact(Params &p, int dtype_index, cudaStream_t st)
     if (per_sm1 < 1 || sms < 1 || maxc < 1) return SPEC_ECUDA;
     const int64_t blocks1 =
         std::max<int64_t>(1, std::min<int64_t>(static_cast<int64_t>(per_sm1) * sms, ceil_div(p.nA, kWarps)));
+    if (prep_pass1(p, blocks1, st) != SPEC_OK) return SPEC_ECUDA;
     k_pass1<Tag, kTreeStochastic, 2><<<static_cast<unsigned>(blocks1), kThreads, kRingBytes, st>>>(p);
     if (cudaGetLastError() != cudaSuccess) return SPEC_ECUDA;
     const int ncl = std::min(maxc, p.B);
@@ -430,6 +443,32 @@ int launch_greedy(Params &p, cudaStream_t st, int dtype_index)
     if (cudaLaunchKernelEx(&cfg, k_greedy_cluster<Tag, kGreedyCluster>, p, slice) != cudaSuccess)
         return SPEC_ECUDA;
     return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ECUDA;
+}
+
+// The workspace form of greedy verification: k_pass1 in the greedy tree
+// mode over the k + 1 target rows of each request, then k_greedy_decide as
+// its programmatic dependent.
+template <class Tag>
+int launch_greedy_streamed(Params &p, int dtype_index, cudaStream_t st)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SPEC_ECUDA;
+    constexpr int kMin1 = pass1_min_blocks<Tag, kTreeGreedy>();
+    int per_sm1, sms;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        per_sm1 = blocks_per_sm(g_pass1_blocks[dev][dtype_index][kTreeGreedy], k_pass1<Tag, kTreeGreedy, kMin1>,
+                                kRingBytes);
+        sms = sm_count(dev);
+    }
+    if (per_sm1 < 1 || sms < 1) return SPEC_ECUDA;
+    const int64_t blocks1 =
+        std::max<int64_t>(1, std::min<int64_t>(static_cast<int64_t>(per_sm1) * sms, ceil_div(p.nA, kWarps)));
+    if (prep_pass1(p, blocks1, st) != SPEC_OK) return SPEC_ECUDA;
+    k_pass1<Tag, kTreeGreedy, kMin1><<<static_cast<unsigned>(blocks1), kThreads, kRingBytes, st>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return SPEC_ECUDA;
+    const int64_t blocksd = std::max<int64_t>(1, std::min<int64_t>(static_cast<int64_t>(4) * sms, p.B));
+    return launch_dependent(k_greedy_decide<Tag>, blocksd, 0, st, p);
 }
 
 void base_params(Params &p, const void *tl, const void *dl, int64_t stride, int B, int V,
@@ -574,7 +613,8 @@ extern "C" int spec_verify_debug_wait_expiry(const void *target_logits, const vo
 extern "C" int spec_verify_greedy(const void *target_logits, spec_dtype_t dtype,
                                   int64_t row_stride, const int32_t *draft_tokens, int batch,
                                   int k, int vocab, int32_t *out_tokens, int32_t *accepted_len,
-                                  int32_t *status, cudaStream_t stream)
+                                  int32_t *status, void *workspace, size_t workspace_bytes,
+                                  cudaStream_t stream)
 {
     if (batch < 0 || k < 1) return SPEC_EINVAL;
     if (k > SPEC_MAX_K) return SPEC_EUNSUPPORTED;
@@ -591,7 +631,20 @@ extern "C" int spec_verify_greedy(const void *target_logits, spec_dtype_t dtype,
     p.out = out_tokens;
     p.acc = accepted_len;
     p.status = status;
-    return dtype == SPEC_BF16 ? launch_greedy<Bf16>(p, stream, 1) : launch_greedy<F32>(p, stream, 0);
+    if (!workspace)
+        return dtype == SPEC_BF16 ? launch_greedy<Bf16>(p, stream, 1) : launch_greedy<F32>(p, stream, 0);
+    // the workspace form: pass 1 as a greedy tree whose N = k + 1 nodes are
+    // the target rows, then the linear decide step
+    const Layout L = layout(batch, k + 1, vocab);
+    if (!L.ok) return SPEC_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 || workspace_bytes < L.total)
+        return SPEC_EWORKSPACE;
+    p.N = k + 1;
+    rc = setup_items(p, k + 1, dtype, false);
+    if (rc != SPEC_OK) return rc;
+    fill_workspace(p, workspace, L);
+    return dtype == SPEC_BF16 ? launch_greedy_streamed<Bf16>(p, 1, stream)
+                              : launch_greedy_streamed<F32>(p, 0, stream);
 }
 
 extern "C" int spec_verify_tree(const void *target_logits, const void *draft_logits,

@@ -84,70 +84,6 @@ __device__ __forceinline__ void merge_row_lane(const Params &p, Load part, float
     S = nan ? __longlong_as_double(0x7FF8000000000000ll) : s;
 }
 
-// The streamer of the fused kernel.  Items [0, nAs) are taken in static
-// round robin (as in pass1_stream); the rest, in chunks of kDynChunk
-// consecutive items from a shared counter, claimed one chunk ahead just
-// before the warp needs it, so the SMs that run faster take more of the
-// tail.  Lane q holds the item id of slot q (kNoItem: the sequence ended).
-constexpr unsigned kDynChunk = 4;
-template <class Tag>
-__device__ __forceinline__ void fused_stream(const Params &p, uint4 *ring, unsigned w, unsigned W)
-{
-    constexpr int kSlot = Pass1Shape<Tag>::kSlot;
-    const int lane = threadIdx.x & 31;
-    unsigned st = w;                  // next static item
-    unsigned dyn = 0, dyn_end = 0;    // current claimed chunk
-    unsigned claim = 0;               // lane 0: the chunk claimed ahead
-    bool claimed = false, done = false;
-    auto claim_ahead = [&]() {
-        if (lane == 0) claim = atomicAdd(p.a_claim, 1u) + 1u;  // the counter starts at all ones
-        claimed = true;
-    };
-    auto next_item = [&]() -> unsigned {
-        if (st < p.nAs) {
-            const unsigned it = st;
-            st += W;
-            if (st >= p.nAs) claim_ahead();  // the next item comes from a claim
-            return it;
-        }
-        if (dyn == dyn_end) {
-            if (!claimed) claim_ahead();
-            const unsigned c = __shfl_sync(kFull, claim, 0);
-            claimed = false;
-            const unsigned first = p.nAs + kDynChunk * c;
-            if (c >= (p.nA - p.nAs + kDynChunk - 1) / kDynChunk || first >= p.nA) {
-                done = true;
-                return kNoItem;
-            }
-            dyn = first;
-            dyn_end = min(first + kDynChunk, p.nA);
-            claim_ahead();
-        }
-        return dyn++;
-    };
-    unsigned meta = kNoItem;
-    auto refill = [&](int q) {
-        const unsigned it = done ? kNoItem : next_item();
-        if (it != kNoItem) issue_item<Tag>(item1<Tag, kLinear>(p, it, false), ring + q * kSlot);
-        if (lane == q) meta = it;
-        commit_copies();
-    };
-#pragma unroll 1
-    for (int q = 0; q < kRing1; ++q) refill(q);
-    int q = 0;
-#pragma unroll 1
-    for (;;) {
-        wait_copies<kRing1 - 1>();
-        const unsigned it = __shfl_sync(kFull, meta, q);
-        if (it == kNoItem) break;
-        const int s = static_cast<int>(it - fdiv(it, p.div_s) * static_cast<unsigned>(p.S));
-        reduce_item1<Tag, kLinear>(p, it, s, ring + q * kSlot);
-        refill(q);
-        q = (q + 1 == kRing1) ? 0 : q + 1;
-    }
-    wait_copies<0>();
-}
-
 // The decide task of request b: wait until all its pass-1 partials are
 // stored, merge its rows (a lane per row), decide, publish.  scr: the
 // warp's region; R*S partials are staged there when they fit, else
@@ -304,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_fused(const __grid_constant__ P
     const int warp = threadIdx.x >> 5;
     uint4 *region = fdyn + warp * kRegion;
     if (warp < kStreamers)
-        fused_stream<Tag>(p, region, blockIdx.x * kStreamers + warp, gridDim.x * kStreamers);
+        pass1_stream<Tag, kLinear>(p, region, blockIdx.x * kStreamers + warp, gridDim.x * kStreamers);
     fused_tasks<Tag>(p, region, tab);
 }
 

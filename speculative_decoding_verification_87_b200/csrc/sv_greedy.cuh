@@ -1,19 +1,27 @@
-// sv_greedy.cuh -- greedy (argmax-match) verification without workspace.
+// sv_greedy.cuh -- greedy (argmax-match) verification.
 //
 // "Accelerating Sonar through speculation", section "Target-Draft": the
 // draft emits its top token at each step, so a draft is kept exactly when it
 // equals the target's top token; at the first mismatch (or after all k) the
 // target's top token is emitted.
 //
-// One thread-block cluster owns a request at a time: each of its CL blocks
-// reduces one contiguous slice of each of the k+1 target rows to (max,
-// lowest argmax, NaN seen) in its shared memory; after a cluster barrier the
-// rank-0 block merges the CL partials through distributed shared memory,
-// scans for the first mismatch and writes the outputs.  Partials are double
-// buffered and the cluster barrier is split (arrive, then wait): only rank 0
-// waits at the end of a request, the other blocks go on to the next one.
-// Clusters stride over the batch; a block's reads run one step ahead of its
-// reductions and barriers.
+// Two forms with identical outputs:
+//
+//  * With a workspace: pass 1 streams every target row as the greedy tree
+//    mode does (k_pass1: (max, lowest argmax, NaN seen) per 2048-entry item,
+//    stored as partials), then k_greedy_decide merges each row's partials
+//    and scans for the first mismatch, a block per request.
+//
+//  * Without a workspace (k_greedy_cluster): one thread-block cluster owns a
+//    request at a time; each of its CL blocks reduces one contiguous slice of
+//    each of the k+1 rows in its shared memory, a block's reads running one
+//    step ahead of its reductions.  The cluster merge is pipelined by one
+//    request: at the end of request r a block publishes its partials (double
+//    buffered by request parity) and arrives on the split cluster barrier; at
+//    the end of request r+1 it waits for that phase, and the rank-0 block
+//    merges request r's partials of all CL blocks through distributed shared
+//    memory and writes the outputs.  No block waits for the request it has
+//    just finished.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -80,7 +88,48 @@ __global__ void __launch_bounds__(kThreads) k_greedy_cluster(const Params p, int
     float best = -INFINITY;
     int idx = INT_MAX;
     bool nan = false;
-    int rq = 0;  // requests done by this cluster (parity selects the partials buffer)
+    int rq = 0, prev_b = -1;  // requests done by this cluster; the last one
+    // rank 0: merge request bb's partials (buffer buf) of all blocks and
+    // write its outputs (every thread of the block calls it)
+    auto merge_write = [&](int bb, int buf) {
+        if (tid == 0) nan_sh = 0;
+        __syncthreads();
+        for (int jj = tid; jj <= k; jj += kThreads) {
+            float bv = -INFINITY;
+            int bi = INT_MAX;
+            bool nn = false;
+            for (int r = 0; r < CL; ++r) {  // slices in index order
+                const float2 *rp = cluster.map_shared_rank(&part[buf][0], r);
+                const float2 v = rp[jj];
+                if (v.x != v.x) nn = true;
+                else argmax_take(bv, bi, v.x, __float_as_int(v.y));
+            }
+            if (nn) atomicOr(&nan_sh, 1);
+            g_sh[jj] = (bi == INT_MAX) ? 0 : bi;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            int x = -1;
+            bool tok_ok = true;
+            if (lane < k) {
+                x = __ldg(p.tokens + static_cast<int64_t>(bb) * k + lane);
+                tok_ok = (x >= 0 && x < p.V);
+            }
+            const int bits = (__any_sync(kFull, !tok_ok) ? kStToken : 0) | (nan_sh ? kStLogit : 0);
+            const unsigned mism = __ballot_sync(kFull, lane < k && x != g_sh[lane < k ? lane : 0]);
+            const int n = mism ? __ffs(mism) - 1 : k;
+            int32_t *out = p.out + static_cast<int64_t>(bb) * (k + 1);
+            for (int jj = lane; jj <= k; jj += 32) {
+                int v = -1;
+                if (!bits) v = (jj < n) ? x : (jj == n ? g_sh[n] : -1);  // jj < n implies jj == lane
+                out[jj] = v;
+            }
+            if (lane == 0) {
+                p.acc[bb] = bits ? -1 : n;
+                report(p.status, bits);
+            }
+        }
+    };
 #pragma unroll 1
     while (b < p.B) {
         // the step after this one
@@ -134,6 +183,12 @@ __global__ void __launch_bounds__(kThreads) k_greedy_cluster(const Params p, int
             nan = false;
             if (j == k) {  // the request is reduced in every warp of the block
                 __syncthreads();
+                // phase rq-1 (the previous request) is complete in every
+                // block: rank 0 merges it now
+                if (rq > 0) {
+                    cluster_wait();
+                    if (rank == 0) merge_write(prev_b, buf ^ 1);
+                }
                 for (int jj = tid; jj <= k; jj += kThreads) {
                     float bv = -INFINITY;
                     int bi = INT_MAX;
@@ -146,51 +201,8 @@ __global__ void __launch_bounds__(kThreads) k_greedy_cluster(const Params p, int
                     }
                     part[buf][jj] = make_float2(nn ? __int_as_float(0x7FC00000) : bv, __int_as_float(bi));
                 }
-                // split cluster barrier: every block arrives once its partials
-                // are in place; only rank 0 waits here (it reads them all), the
-                // others wait for this phase just before their next arrival
-                if (rq > 0 && rank != 0) cluster_wait();
-                cluster_arrive();
-                if (rank == 0) {
-                    cluster_wait();
-                    if (tid == 0) nan_sh = 0;
-                    __syncthreads();
-                    for (int jj = tid; jj <= k; jj += kThreads) {
-                        float bv = -INFINITY;
-                        int bi = INT_MAX;
-                        bool nn = false;
-                        for (int r = 0; r < CL; ++r) {  // slices in index order
-                            const float2 *rp = cluster.map_shared_rank(&part[buf][0], r);
-                            const float2 v = rp[jj];
-                            if (v.x != v.x) nn = true;
-                            else argmax_take(bv, bi, v.x, __float_as_int(v.y));
-                        }
-                        if (nn) atomicOr(&nan_sh, 1);
-                        g_sh[jj] = (bi == INT_MAX) ? 0 : bi;
-                    }
-                    __syncthreads();
-                    if (warp == 0) {
-                        int x = -1;
-                        bool tok_ok = true;
-                        if (lane < k) {
-                            x = __ldg(p.tokens + static_cast<int64_t>(b) * k + lane);
-                            tok_ok = (x >= 0 && x < p.V);
-                        }
-                        const int bits = (__any_sync(kFull, !tok_ok) ? kStToken : 0) | (nan_sh ? kStLogit : 0);
-                        const unsigned mism = __ballot_sync(kFull, lane < k && x != g_sh[lane < k ? lane : 0]);
-                        const int n = mism ? __ffs(mism) - 1 : k;
-                        int32_t *out = p.out + static_cast<int64_t>(b) * (k + 1);
-                        for (int jj = lane; jj <= k; jj += 32) {
-                            int v = -1;
-                            if (!bits) v = (jj < n) ? x : (jj == n ? g_sh[n] : -1);  // jj < n implies jj == lane
-                            out[jj] = v;
-                        }
-                        if (lane == 0) {
-                            p.acc[b] = bits ? -1 : n;
-                            report(p.status, bits);
-                        }
-                    }
-                }
+                cluster_arrive();  // phase rq: this block's partials of request b are in place
+                prev_b = b;
                 ++rq;
             }
         }
@@ -200,11 +212,75 @@ __global__ void __launch_bounds__(kThreads) k_greedy_cluster(const Params p, int
         j = nj;
         it = nit;
     }
-    // the last phase: rank 0 has waited on it; the others wait now, then one
-    // full barrier so that no block leaves while rank 0 may still read its
+    // the last request: wait for its phase and merge it; then one full
+    // barrier so that no block leaves while rank 0 may still read its
     // partials
-    if (rq > 0 && rank != 0) cluster_wait();
+    if (rq > 0) {
+        cluster_wait();
+        if (rank == 0) merge_write(prev_b, (rq - 1) & 1);
+    }
     cluster.sync();
+}
+
+// The decide step of the workspace form: a block per request (blocks stride
+// over the batch), a warp per row (rows w, w + kWarps, ...).  A row's S
+// pass-1 partials are merged lane-strided and then across the warp;
+// argmax_take breaks ties by the lower index, so the result is the lowest
+// argmax whatever the merge order.  Warp 0 then scans for the first
+// mismatch.  The draft tokens are inputs and are read before pass 1 ends.
+template <class Tag>
+__global__ void __launch_bounds__(kThreads) k_greedy_decide(const __grid_constant__ Params p)
+{
+    __shared__ int g_sh[kMaxRowsGreedy];
+    __shared__ int bits_sh;
+    const int k = p.k, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int b = blockIdx.x;
+    auto token = [&](int bb) {
+        return (bb < p.B && lane < k) ? __ldg(p.tokens + static_cast<int64_t>(bb) * k + lane) : -1;
+    };
+    int x = warp == 0 ? token(b) : -1;
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    for (; b < p.B; b += gridDim.x) {
+        if (tid == 0) bits_sh = 0;
+        __syncthreads();
+        for (int r = warp; r <= k; r += kWarps) {
+            const float2 *pp = p.rowpart + (static_cast<int64_t>(b) * (k + 1) + r) * p.S;
+            float bv = -INFINITY;
+            int bi = INT_MAX;
+            bool nan = false;
+            for (int s = lane; s < p.S; s += 32) {
+                const float2 v = __ldcg(pp + s);
+                if (v.x != v.x) nan = true;
+                else argmax_take(bv, bi, v.x, __float_as_int(v.y));
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ov = __shfl_xor_sync(kFull, bv, o);
+                const int oi = __shfl_xor_sync(kFull, bi, o);
+                argmax_take(bv, bi, ov, oi);
+            }
+            if (__any_sync(kFull, nan) && lane == 0) atomicOr(&bits_sh, kStLogit);
+            if (lane == 0) g_sh[r] = (bi == INT_MAX) ? 0 : bi;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            const bool tok_ok = lane >= k || (x >= 0 && x < p.V);
+            const int bits = (__any_sync(kFull, !tok_ok) ? kStToken : 0) | bits_sh;
+            const unsigned mism = __ballot_sync(kFull, lane < k && x != g_sh[lane < k ? lane : 0]);
+            const int n = mism ? __ffs(mism) - 1 : k;
+            int32_t *out = p.out + static_cast<int64_t>(b) * (k + 1);
+            for (int jj = lane; jj <= k; jj += 32) {
+                int v = -1;
+                if (!bits) v = (jj < n) ? x : (jj == n ? g_sh[n] : -1);  // jj < n implies jj == lane
+                out[jj] = v;
+            }
+            if (lane == 0) {
+                p.acc[b] = bits ? -1 : n;
+                report(p.status, bits);
+            }
+            x = token(b + gridDim.x);
+        }
+    }
 }
 
 }  // namespace sv

@@ -322,31 +322,36 @@ __device__ __forceinline__ void reduce_item1(const Params &p, unsigned item, int
     }
     float2 part;
     if (MODE == kTreeGreedy) {
-        float best = -INFINITY;
+        // the item's max from packed maxima (NaN if any entry is NaN), then
+        // the lowest index holding it: entry e of lane l's vector v is entry
+        // (v * 32 + l) * kVec + e of the item, so the first vector round
+        // with a hit, its lowest lane and that lane's first entry give it
+        const float M = warp_max_nan(lane_max<Tag>(raw));
         int idx = INT_MAX;
-        bool nan = false;
+        bool found = !(M == M && M != -INFINITY);  // NaN or all -inf: no search
+        // fully unrolled with a warp-uniform guard (no break), so that raw[]
+        // stays in registers
 #pragma unroll
         for (int v = 0; v < kV; ++v) {
-            float x[kVec];
-            unpack<Tag>(raw[v], x);
-            const int e0 = e_begin + (v * 32 + lane) * kVec;
+            if (found) continue;
+            const unsigned hit = __ballot_sync(kFull, vec_max<Tag>(raw[v]) == M);
+            if (hit) {
+                const int w = __ffs(hit) - 1;
+                int first = 0;
+                if (lane == w) {
+                    float x[kVec];
+                    unpack<Tag>(raw[v], x);
+                    first = kVec - 1;
 #pragma unroll
-            for (int e = 0; e < kVec; ++e) {
-                nan |= (x[e] != x[e]);
-                if (x[e] > best) {
-                    best = x[e];
-                    idx = e0 + e;
+                    for (int e = kVec - 1; e >= 0; --e)
+                        if (x[e] == M) first = e;
                 }
+                first = __shfl_sync(kFull, first, w);
+                idx = e_begin + (v * 32 + w) * kVec + first;
+                found = true;
             }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(kFull, best, o);
-            const int oi = __shfl_xor_sync(kFull, idx, o);
-            argmax_take(best, idx, ov, oi);
-        }
-        nan = __any_sync(kFull, nan);
-        part = make_float2(nan ? __int_as_float(0x7FC00000) : best, __int_as_float(idx));
+        part = make_float2(M, __int_as_float(idx));
     } else {
         const float c = p.c;
         const float m = lane_max<Tag>(raw);
@@ -373,42 +378,82 @@ __device__ __forceinline__ void reduce_item1(const Params &p, unsigned item, int
     if (lane == 0 && !p.diag_no_partials) __stcg(p.rowpart + item, part);
 }
 
-// The pass-1 worker: warp w of W takes items w, w + W, w + 2W, ... (items
-// are equal, so a static round robin balances them without any shared
-// counter), copied into a kRing1-slot ring kRing1 - 1 items ahead of their
-// reduction.  Lane q holds whether the item of slot q is read at all, so
-// the loop body exists once with a rotating slot index.
+// The pass-1 worker.  Items [0, nAs) are taken in static round robin (warp
+// w of W takes w, w + W, ...: items are equal, so this balances them
+// without a shared counter); the rest, in chunks of kDynChunk consecutive
+// items from a counter (a_claim, all ones at the start of a call), claimed
+// one chunk ahead just before the warp needs it, so that the SMs that run
+// faster take more of the tail.  Items are copied into a kRing1-slot ring
+// kRing1 - 1 items ahead of their reduction; lane q holds the item of slot
+// q (kNoItem: the sequence ended) and whether it is read at all (tree
+// draft rows of leaves are not), so the loop body exists once with a
+// rotating slot index.
+constexpr unsigned kDynChunk = 4;
 template <class Tag, int MODE>
 __device__ __forceinline__ void pass1_stream(const Params &p, uint4 *ring, unsigned w, unsigned W)
 {
     constexpr int kSlot = Pass1Shape<Tag>::kSlot;
     const int lane = threadIdx.x & 31;
-    bool act = true;  // lane q: the item in slot q is read
-    unsigned next = w;  // the next item to copy
-    auto refill = [&](int q) {
-        if (next < p.nA) {
-            const Item1 it = item1<Tag, MODE>(p, next);
-            issue_item<Tag>(it, ring + q * kSlot);
-            if (lane == q) act = it.active;
+    unsigned st = w;                  // next static item
+    unsigned dyn = 0, dyn_end = 0;    // current claimed chunk
+    unsigned claim = 0;               // lane 0: the chunk claimed ahead
+    bool claimed = false, done = false;
+    auto claim_ahead = [&]() {
+        if (lane == 0) claim = atomicAdd(p.a_claim, 1u) + 1u;  // the counter starts at all ones
+        claimed = true;
+    };
+    auto next_item = [&]() -> unsigned {
+        if (st < p.nAs) {
+            const unsigned it = st;
+            st += W;
+            if (st >= p.nAs) claim_ahead();  // the next item comes from a claim
+            return it;
         }
-        next += W;
+        if (dyn == dyn_end) {
+            if (!claimed) claim_ahead();
+            const unsigned c = __shfl_sync(kFull, claim, 0);
+            claimed = false;
+            const unsigned first = p.nAs + kDynChunk * c;
+            if (c >= (p.nA - p.nAs + kDynChunk - 1) / kDynChunk || first >= p.nA) {
+                done = true;
+                return kNoItem;
+            }
+            dyn = first;
+            dyn_end = min(first + kDynChunk, p.nA);
+            claim_ahead();
+        }
+        return dyn++;
+    };
+    unsigned meta = kNoItem;
+    bool act = true;
+    auto refill = [&](int q) {
+        const unsigned it = done ? kNoItem : next_item();
+        bool a = false;
+        if (it != kNoItem) {
+            const Item1 i1 = item1<Tag, MODE>(p, it, MODE != kLinear);
+            issue_item<Tag>(i1, ring + q * kSlot);
+            a = i1.active;
+        }
+        if (lane == q) {
+            meta = it;
+            act = a;
+        }
         commit_copies();
     };
 #pragma unroll 1
     for (int q = 0; q < kRing1; ++q) refill(q);
-    // segment of the item in hand, advanced by W mod S per item
-    int s = static_cast<int>(w - fdiv(w, p.div_s) * static_cast<unsigned>(p.S));
-    const int ws = static_cast<int>(W - fdiv(W, p.div_s) * static_cast<unsigned>(p.S));
     int q = 0;
 #pragma unroll 1
-    for (unsigned item = w; item < p.nA; item += W) {
+    for (;;) {
         wait_copies<kRing1 - 1>();
-        if (MODE == kLinear || __shfl_sync(kFull, act ? 1 : 0, q))
-            reduce_item1<Tag, MODE>(p, item, s, ring + q * kSlot);
+        const unsigned it = __shfl_sync(kFull, meta, q);
+        if (it == kNoItem) break;
+        if (MODE == kLinear || __shfl_sync(kFull, act ? 1 : 0, q)) {
+            const int s = static_cast<int>(it - fdiv(it, p.div_s) * static_cast<unsigned>(p.S));
+            reduce_item1<Tag, MODE>(p, it, s, ring + q * kSlot);
+        }
         refill(q);
         q = (q + 1 == kRing1) ? 0 : q + 1;
-        s += ws;
-        if (s >= p.S) s -= p.S;
     }
     wait_copies<0>();
 }

@@ -137,10 +137,17 @@ def test_greedy_and_tree_host_validation(lib):
     g = lambda **kw: lib.spec_verify_greedy(P(kw.get("tl", 0x1000)), kw.get("dtype", 0),
                                             kw.get("stride", 64), P(0x2000), kw.get("batch", 3),
                                             kw.get("k", 2), kw.get("vocab", 50), P(0x3000),
-                                            P(0x4000), None, None)
+                                            P(0x4000), None, P(kw.get("ws", 0)),
+                                            kw.get("ws_bytes", 0), None)
     assert g(k=0) == SPEC_EINVAL and g(k=40) == SPEC_EUNSUPPORTED
     assert g(stride=63) == SPEC_EALIGN and g(vocab=65) == SPEC_EINVAL
     assert g(batch=0) == SPEC_OK
+    # the streamed form: an aligned workspace of spec_verify_workspace_size(B, k+1, V) bytes
+    need = lib.spec_verify_workspace_size(3, 3, 50)
+    assert need > 0
+    assert g(ws=0x10000, ws_bytes=need - 1) == SPEC_EWORKSPACE
+    assert g(ws=0x10010, ws_bytes=need) == SPEC_EWORKSPACE   # not 256-byte aligned
+    assert g(ws=0x10000, ws_bytes=need, batch=0) == SPEC_OK
 
     def t(**kw):
         return lib.spec_verify_tree(P(0x1000), P(kw.get("dl", 0x2000)), 1, 64, P(0x3000),

@@ -19,10 +19,14 @@ def sv():
     return binding
 
 
-def run_greedy(sv, target, tokens, vocab):
+# the two forms of spec_verify_greedy: streamed (workspace) and cluster (none)
+FORMS = pytest.mark.parametrize("workspace_free", [False, True], ids=["streamed", "cluster"])
+
+
+def run_greedy(sv, target, tokens, vocab, workspace_free=False):
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     out, acc = sv.spec_verify_greedy(to_device(target), to_device(tokens.astype(np.int32)), vocab,
-                                     status=status)
+                                     status=status, workspace_free=workspace_free)
     torch.cuda.synchronize()
     return out.cpu().numpy(), acc.cpu().numpy(), int(status.item())
 
@@ -41,9 +45,10 @@ def run_tree(sv, w, stochastic, seed=0, offset=0, target=None, draft=None):
     return out.cpu().numpy(), acc.cpu().numpy(), path.cpu().numpy(), int(status.item())
 
 
-def test_greedy_full_size_bit_exact(sv, orc):
+@FORMS
+def test_greedy_full_size_bit_exact(sv, orc, workspace_free):
     w = wl.config_greedy(seed=0)
-    out, acc, st = run_greedy(sv, w.target, w.tokens, w.vocab)
+    out, acc, st = run_greedy(sv, w.target, w.tokens, w.vocab, workspace_free)
     o = orc.verify_greedy(w.target, w.tokens, w.vocab)
     assert st == 0
     assert np.array_equal(out, o["out"]) and np.array_equal(acc, o["acc"])
@@ -53,18 +58,20 @@ def test_greedy_full_size_bit_exact(sv, orc):
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("batch,k,vocab,pad", [(1, 4, 128256, 0), (3, 32, 1000, 5),
                                                (37, 2, 77, 3), (5, 1, 1, 0), (300, 3, 4100, 0)])
-def test_greedy_shapes_bit_exact(sv, orc, dtype, batch, k, vocab, pad):
+@FORMS
+def test_greedy_shapes_bit_exact(sv, orc, dtype, batch, k, vocab, pad, workspace_free):
     w = wl.greedy_linear(seed=batch + k, batch=batch, k=k, vocab=vocab, dtype=dtype, pad=pad)
     t = w.target.copy()
     if t.shape[-1] > vocab:
         t[..., vocab:] = np.uint16(0x7FC0) if dtype == "bf16" else np.float32(np.nan)
-    out, acc, st = run_greedy(sv, t, w.tokens, vocab)
+    out, acc, st = run_greedy(sv, t, w.tokens, vocab, workspace_free)
     o = orc.verify_greedy(t, w.tokens, vocab)
     assert st == 0
     assert np.array_equal(out, o["out"]) and np.array_equal(acc, o["acc"])
 
 
-def test_greedy_ties_and_errors(sv, orc):
+@FORMS
+def test_greedy_ties_and_errors(sv, orc, workspace_free):
     # heavy ties: logits drawn from 3 values, argmax ties resolved to the lowest index
     rng = np.random.default_rng(0)
     B, k, V = 64, 4, 3000
@@ -73,7 +80,7 @@ def test_greedy_ties_and_errors(sv, orc):
     for b in range(B):
         for j in range(k):
             x[b, j] = int(np.argmax(t[b, j])) if rng.random() < 0.8 else int(rng.integers(V))
-    out, acc, st = run_greedy(sv, t, x, V)
+    out, acc, st = run_greedy(sv, t, x, V, workspace_free)
     o = orc.verify_greedy(t, x, V)
     assert np.array_equal(out, o["out"]) and np.array_equal(acc, o["acc"])
     # NaN logits and bad tokens
@@ -81,14 +88,14 @@ def test_greedy_ties_and_errors(sv, orc):
     t2[3, 2, 17] = np.nan
     x2 = x.copy()
     x2[5, 0] = V
-    out, acc, st = run_greedy(sv, t2, x2, V)
+    out, acc, st = run_greedy(sv, t2, x2, V, workspace_free)
     o = orc.verify_greedy(t2, x2, V)
     assert st == (1 | 4)
     assert np.array_equal(out, o["out"]) and np.array_equal(acc, o["acc"])
     # a fully -inf row: argmax is index 0
     t3 = t.copy()
     t3[7, 0, :] = -np.inf
-    out, acc, st = run_greedy(sv, t3, x, V)
+    out, acc, st = run_greedy(sv, t3, x, V, workspace_free)
     o = orc.verify_greedy(t3, x, V)
     assert st == 0 and np.array_equal(out, o["out"])
 
