@@ -2,7 +2,8 @@
 //
 // spec_verify_linear: one memset of the call's counters and pass-1
 // partials, then a cooperative launch of the persistent kernel k_fused
-// (sv_fused.cuh).
+// (sv_fused.cuh); batches of one or two requests take the four-kernel path
+// of the tree calls instead (pass 1, decide, pass 2, finalize).
 // spec_verify_tree: the pass-1 kernel, the decide kernel and, where a token
 // is drawn, the pass-2 and finalize kernels (sv_verify.cuh), each a
 // programmatic dependent of the one before.
@@ -534,6 +535,9 @@ extern "C" const char *spec_verify_strerror(int code)
 
 namespace {
 
+// Batches up to this size take the four-kernel linear path.
+constexpr int kFourKernelMaxBatch = 2;
+
 // spec_verify_linear, with the diagnostic switches of
 // spec_verify_debug_wait_expiry (poll_limit 0: the normal limit).
 int linear_call(const void *target_logits, const void *draft_logits, spec_dtype_t dtype,
@@ -576,6 +580,12 @@ int linear_call(const void *target_logits, const void *draft_logits, spec_dtype_
     rc = setup_items(p, R, dtype, true);
     if (rc != SPEC_OK) return rc;
     fill_workspace(p, workspace, L);
+    // one or two requests leave the one-kernel path nothing to overlap (no
+    // later request streams while an earlier one draws): the four
+    // programmatic-dependent kernels, each over the whole GPU, finish first
+    if (batch <= kFourKernelMaxBatch && !diag)
+        return dtype == SPEC_BF16 ? launch_verify<Bf16, kLinear>(p, L, workspace, 1, stream)
+                                  : launch_verify<F32, kLinear>(p, L, workspace, 0, stream);
     return dtype == SPEC_BF16 ? launch_fused<Bf16>(p, L, workspace, 1, stream)
                               : launch_fused<F32>(p, L, workspace, 0, stream);
 }

@@ -50,6 +50,14 @@ __device__ __forceinline__ unsigned long long ld_poll64(const void *p)
     return __ldcv(reinterpret_cast<const unsigned long long *>(p));
 }
 __device__ __forceinline__ unsigned ld_poll32(const unsigned *p) { return __ldcv(p); }
+// A flag read with acquire semantics: this thread's later reads see what the
+// writer stored before its release (a fence, then the flag).
+__device__ __forceinline__ unsigned ld_acquire32(const unsigned *p)
+{
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
 
 __device__ __forceinline__ void backoff(unsigned &ns)
 {
@@ -99,8 +107,18 @@ __device__ __forceinline__ bool decide_task(const Params &p, int b, uint4 *scr)
     const bool staged = static_cast<size_t>(n) * sizeof(float2) + sizeof(double) * 2 * 65 <=
                         sizeof(uint4) * kRegion;
     bool done = false;
-    unsigned ns = 64;
-    for (unsigned it = 0; it < p.poll_limit; ++it) {
+    unsigned ns = 64, it = 0;
+    // the request's last partial first, one word per poll (items are taken
+    // in increasing order, so it is among the last of the request's to be
+    // stored); then every partial until all are stored
+    for (; it < p.poll_limit; ++it) {
+        unsigned seen = 0;
+        if (lane == 0) seen = static_cast<unsigned>(ld_poll64(part + n - 1)) != kPartEmpty;
+        if (__shfl_sync(kFull, seen, 0)) break;
+        backoff(ns);
+    }
+    ns = 64;
+    for (; it < p.poll_limit; ++it) {
         bool all = true;
         for (int i = lane; i < n; i += 32) {
             const unsigned long long v = ld_poll64(part + i);
@@ -152,43 +170,45 @@ __device__ __forceinline__ bool decide_task(const Params &p, int b, uint4 *scr)
     return true;
 }
 
-// Wait (lane 0 polls, bounded) until request b is decided; then a fence
-// orders the request record's reads after the flag.  False on expiry.
-__device__ __forceinline__ bool wait_decided(const Params &p, int b)
+// Request b's decision, published?  Every lane reads the flag with acquire
+// semantics, so the request record read afterwards is the published one.
+__device__ __forceinline__ bool is_decided(const Params &p, int b)
 {
-    int ok = 0;
-    if ((threadIdx.x & 31) == 0) {
-        unsigned ns = 32;
-        for (unsigned i = 0; i < p.poll_limit; ++i) {
-            if (ld_poll32(&p.decided[b]) == 1u) {
-                ok = 1;
-                break;
-            }
-            backoff(ns);
-        }
-        if (ok) __threadfence();
-        else report(p.status, kStTimeout);
-    }
-    return __shfl_sync(kFull, ok, 0) != 0;
+    return __all_sync(kFull, ld_acquire32(&p.decided[b]) == 1u);
 }
 
-// The task worker: tasks in request order from the shared counter (which
-// starts at kPartEmpty, so a claim returns the task id minus one).
+// Wait (bounded) until request b is decided.  False on expiry.
+__device__ __forceinline__ bool wait_decided(const Params &p, int b)
+{
+    unsigned ns = 32;
+    for (unsigned i = 0; i < p.poll_limit; ++i) {
+        if (is_decided(p, b)) return true;
+        backoff(ns);
+    }
+    if ((threadIdx.x & 31) == 0) report(p.status, kStTimeout);
+    return false;
+}
+
+// The task worker.  Tasks come in request order from one shared counter
+// (which starts at kPartEmpty, so a claim returns the task id minus one):
+// first the B decide tasks, then the B * S2 pass-2 items.  A decide task is
+// claimed only by a free warp, so it starts at once and no item waits on a
+// decide that waits on that item's warp.  Once a warp's claim is an item,
+// every decide has been claimed, and the warp claims one item ahead: the
+// next item is staged (if its request is decided by then) while the
+// current one is reduced.
 template <class Tag>
 __device__ __forceinline__ void fused_tasks(const Params &p, uint4 *region, const double *tab)
 {
+    constexpr int kBuf = StageShape<Tag>::kPerBuf;
     const int lane = threadIdx.x & 31;
-    // one staging buffer (an item is staged and reduced in turn), then the
-    // finalize scratch
-    static_assert(StageShape<Tag>::kPerBuf <= kRegion, "a staging buffer fits a warp region");
-    uint4 *stage = region;
-    double *W_sh = reinterpret_cast<double *>(region + StageShape<Tag>::kPerBuf);
+    // two staging buffers, then the finalize scratch
+    static_assert(2 * kBuf <= kRegion, "two staging buffers fit a warp region");
+    double *W_sh = reinterpret_cast<double *>(region + 2 * kBuf);
     const bool w_shared = 2 * static_cast<size_t>(p.S2) * sizeof(double) <=
-                          sizeof(uint4) * static_cast<size_t>(kRegion - StageShape<Tag>::kPerBuf);
-    // tasks [0, B): the decide steps; then B * S2 items in request order
-    const unsigned ntask = static_cast<unsigned>(p.B) * (static_cast<unsigned>(p.S2) + 1u);
-    // a task is claimed only by a free warp: a claimed decide task starts at
-    // once, so no item waits on a decide that waits on that item's warp
+                          sizeof(uint4) * static_cast<size_t>(kRegion - 2 * kBuf);
+    const unsigned nB = static_cast<unsigned>(p.B);
+    const unsigned ntask = nB * (static_cast<unsigned>(p.S2) + 1u);
     auto claim = [&]() {
         unsigned t = 0;
         if (lane == 0) t = atomicAdd(p.p2claim, 1u) + 1u;
@@ -196,36 +216,73 @@ __device__ __forceinline__ void fused_tasks(const Params &p, uint4 *region, cons
     };
     unsigned cur = claim();
 #pragma unroll 1
-    while (cur < ntask) {
-        if (cur < static_cast<unsigned>(p.B)) {
-            if (!decide_task<Tag>(p, static_cast<int>(cur), region)) break;
-        } else {
-            const unsigned item = cur - static_cast<unsigned>(p.B);
-            const int b = static_cast<int>(fdiv(item, p.div_s2));
-            const int s2 = static_cast<int>(item - static_cast<unsigned>(b) * static_cast<unsigned>(p.S2));
-            if (!wait_decided(p, b)) break;
-            const ItemInfo it = load_item_info(p, b);
-            if (it.mode == kModeResidual || it.mode == kModeTargetRow) {
-                if (it.mode == kModeResidual) stage_item<Tag, true>(p, it, s2, stage);
-                else stage_item<Tag, false>(p, it, s2, stage);
-                commit_copies();
-                wait_copies<0>();
-                if (it.mode == kModeResidual) p2_item<Tag, true>(p, b, s2, it, stage, tab);
-                else p2_item<Tag, false>(p, b, s2, it, stage, tab);
-                __threadfence();  // every lane's stores of the item precede its arrival
-                __syncwarp();
-                unsigned o = 0;
-                if (lane == 0) {
-                    o = atomicAdd(&p.p2cnt[b], 1u) + 1u;  // the counter starts at kPartEmpty
-                    if (o == static_cast<unsigned>(p.S2) - 1u) __threadfence();
-                }
-                if (__shfl_sync(kFull, o == static_cast<unsigned>(p.S2) - 1u ? 1 : 0, 0)) {
-                    double *W = w_shared ? W_sh : p.p2w + 2 * static_cast<int64_t>(b) * p.S2;
-                    finalize<Tag>(p, b, tab, W, W + p.S2);
-                }
+    while (cur < nB) {
+        if (!decide_task<Tag>(p, static_cast<int>(cur), region)) return;
+        cur = claim();
+    }
+    if (cur >= ntask) return;
+
+    // a held item: request, segment, record; staged = its copies are issued
+    // (one committed group per staged item)
+    struct Held {
+        int b, s2;
+        ItemInfo it;
+        bool staged;
+    };
+    auto locate = [&](unsigned t) {
+        Held h;
+        const unsigned item = t - nB;
+        h.b = static_cast<int>(fdiv(item, p.div_s2));
+        h.s2 = static_cast<int>(item - static_cast<unsigned>(h.b) * static_cast<unsigned>(p.S2));
+        h.it.mode = kModeNone;
+        h.staged = false;
+        return h;
+    };
+    auto stage = [&](Held &h, uint4 *buf) {
+        h.it = load_item_info(p, h.b);
+        if (h.it.mode == kModeResidual) stage_item<Tag, true>(p, h.it, h.s2, buf);
+        else if (h.it.mode == kModeTargetRow) stage_item<Tag, false>(p, h.it, h.s2, buf);
+        commit_copies();
+        h.staged = true;
+    };
+    Held c = locate(cur);
+    if (!wait_decided(p, c.b)) return;
+    stage(c, region);
+    int bc = 0;
+#pragma unroll 1
+    for (;;) {
+        const unsigned nt = claim();
+        const bool more = nt < ntask;
+        Held n = more ? locate(nt) : c;
+        if (more && is_decided(p, n.b)) stage(n, region + (bc ^ 1) * kBuf);
+        const bool ahead = more && n.staged;
+        if (ahead) wait_copies<1>();
+        else wait_copies<0>();
+        const uint4 *buf = region + bc * kBuf;
+        if (c.it.mode == kModeResidual || c.it.mode == kModeTargetRow) {
+            if (c.it.mode == kModeResidual) p2_item<Tag, true>(p, c.b, c.s2, c.it, buf, tab);
+            else p2_item<Tag, false>(p, c.b, c.s2, c.it, buf, tab);
+            // no copy in flight across the fence (a fence waits for them)
+            if (ahead) wait_copies<0>();
+            __threadfence();  // every lane's stores of the item precede its arrival
+            __syncwarp();
+            unsigned o = 0;
+            if (lane == 0) {
+                o = atomicAdd(&p.p2cnt[c.b], 1u) + 1u;  // the counter starts at kPartEmpty
+                if (o == static_cast<unsigned>(p.S2) - 1u) __threadfence();
+            }
+            if (__shfl_sync(kFull, o == static_cast<unsigned>(p.S2) - 1u ? 1 : 0, 0)) {
+                double *W = w_shared ? W_sh : p.p2w + 2 * static_cast<int64_t>(c.b) * p.S2;
+                finalize<Tag>(p, c.b, tab, W, W + p.S2);
             }
         }
-        cur = claim();
+        if (!more) break;
+        if (!n.staged) {
+            if (!wait_decided(p, n.b)) break;
+            stage(n, region + (bc ^ 1) * kBuf);
+        }
+        c = n;
+        bc ^= 1;
     }
     wait_copies<0>();
 }
