@@ -60,8 +60,16 @@ constexpr int kMaxS2Shared = 1024;
 
 // Shared memory of a decide block beside the row statistics (trees).
 struct TreeScratch {
+    int par[kMaxNodes];             // parents as given (checked in tree_prepare)
+    int tok[kMaxNodes];
     short depth[kMaxNodes];
-    unsigned char flag[kMaxNodes];  // 1 has child, 2 test passed, 4 accepted
+    unsigned char flag[kMaxNodes];  // 1 has child, 2 test passed
+    int err;                        // status bits of the request
+    int key;                        // deepest accepted node: depth << 11 | (kMaxNodes - 1 - node)
+};
+// The accept and sample uniforms of a stochastic tree's nodes.
+struct TreeUniforms {
+    double ua[kMaxNodes], us[kMaxNodes];
 };
 // The logits a stochastic tree's node tests read (target and draft row of
 // the parent at the node's token), fetched before pass 1 completes.
@@ -624,135 +632,161 @@ __device__ __forceinline__ void decide_linear(const Params &p, int b, RowStats s
 }
 
 
-// The tree decide step of request b, one warp: checks, node tests (lanes
-// over nodes; stochastic tests read the prefetched logits), then depths and
-// acceptance level by level (at most max_depth + 1 rounds, lanes over
-// nodes), the deepest accepted node by a warp reduction (ties to the
-// lowest index), and the outputs.
+constexpr int kDecideThreads = 1024;
+
+// The tree decide step of request b, in two parts run by every thread of
+// the decide block.
+//
+// tree_prepare reads only inputs, so it runs before pass 1 completes: the
+// parents and tokens (into shared memory), the structural checks (root,
+// parents before children, tokens in range), which nodes have children,
+// every node's depth (a walk up its parents, at most max_depth + 1 steps;
+// a node still short of the root is too deep), and for stochastic trees
+// the logits each node test reads and the Philox uniforms of every test
+// and of every possible draw.
 template <class Tag, int MODE>
-__device__ __forceinline__ void decide_tree(const Params &p, int b, RowStats rs, TreeScratch &sh,
-                                            const TreeProbe *pr)
+__device__ __forceinline__ void tree_prepare(const Params &p, int b, TreeScratch &ts, TreeProbe &tp,
+                                             TreeUniforms &tu)
 {
-    const int lane = threadIdx.x & 31;
-    const int N = p.N, R = p.R;
+    constexpr int kT = kDecideThreads;
+    const int N = p.N, tid = threadIdx.x;
     const int32_t *pa = p.parents + static_cast<int64_t>(b) * N;
     const int32_t *tk = p.tokens + static_cast<int64_t>(b) * N;
-    int err = 0;  // sh.flag holds "has a child" (bit 1), set by the block
-    for (int i = lane; i < N; i += 32) {
-        const int par = __ldg(pa + i);
-        sh.depth[i] = i == 0 ? 0 : -1;
+    if (tid == 0) {
+        ts.err = 0;
+        ts.key = 0;
+    }
+    for (int i = tid; i < N; i += kT) {
+        ts.par[i] = __ldg(pa + i);
+        ts.tok[i] = __ldg(tk + i);
+        ts.flag[i] = 0;
+    }
+    __syncthreads();
+    int err = 0;
+    for (int i = tid; i < N; i += kT) {
+        const int par = ts.par[i], t = ts.tok[i];
         if (i == 0) {
             if (par != -1) err |= kStTree;
         } else if (par < 0 || par >= i) {
             err |= kStTree;
         } else {
-            const int t = __ldg(tk + i);
+            ts.flag[par] = 1;  // every writer stores 1
             if (t < 0 || t >= p.V) err |= kStToken;
         }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) err |= __shfl_xor_sync(kFull, err, o);
-    __syncwarp();
-    if (!(err & kStTree)) {
-        // depth of every node: its parent's plus one, settled one level per
-        // round; a node still unset after max_depth + 1 rounds is too deep
-        for (int round = 0; round <= p.max_depth; ++round) {
-            for (int i = 1 + lane; i < N; i += 32) {
-                if (sh.depth[i] >= 0) continue;
-                const int dp = sh.depth[__ldg(pa + i)];
-                if (dp >= 0) sh.depth[i] = static_cast<short>(dp + 1);
+        if (MODE == kTreeStochastic) {
+            float lt = 0.f, ld = 0.f;
+            if (i > 0 && par >= 0 && par < i && t >= 0 && t < p.V) {
+                const int64_t off = (static_cast<int64_t>(b) * N + par) * p.stride + t;
+                lt = load_logit<Tag>(p.tl, off);
+                ld = load_logit<Tag>(p.dl, off);
             }
-            __syncwarp();
+            tp.lt[i] = lt;
+            tp.ld[i] = ld;
+            if (i > 0)
+                tu.ua[i] = philox_uniform(p.seed, static_cast<uint32_t>(b), static_cast<uint32_t>(i - 1),
+                                          kPurposeAccept, p.offset);
+            tu.us[i] = philox_uniform(p.seed, static_cast<uint32_t>(b), static_cast<uint32_t>(i),
+                                      kPurposeSample, p.offset);
         }
-        bool deep = false;
-        for (int i = lane; i < N; i += 32) deep |= sh.depth[i] < 0 || sh.depth[i] > p.max_depth;
-        if (__any_sync(kFull, deep)) err |= kStTree;
     }
+    if (err) atomicOr(&ts.err, err);
+    __syncthreads();
+    if (!(ts.err & kStTree)) {
+        for (int i = tid; i < N; i += kT) {
+            int j = i, d = 0;
+            while (j != 0 && d <= p.max_depth) {
+                j = ts.par[j];
+                ++d;
+            }
+            const bool ok = (j == 0);
+            ts.depth[i] = static_cast<short>(ok ? d : -1);
+            if (!ok) atomicOr(&ts.err, kStTree);
+        }
+    }
+    __syncthreads();
+}
 
-    // rows the mode reads must be usable: every target row, and the draft
-    // rows of nodes with children
+// tree_decide runs once the rows are merged: the row checks (every target
+// row, and the draft rows of nodes with children), the node tests (a thread
+// per node; greedy: the token is the parent's argmax; stochastic: the
+// acceptance test), acceptance (a node is accepted when every node on its
+// path passed its test: a walk up at most max_depth parents), the deepest
+// accepted node (ties to the lowest index), and the outputs.
+template <class Tag, int MODE>
+__device__ __forceinline__ void tree_decide(const Params &p, int b, RowStats rs, TreeScratch &ts,
+                                            const TreeProbe &tp, const TreeUniforms &tu)
+{
+    constexpr int kT = kDecideThreads;
+    const int N = p.N, R = p.R, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     bool bad = false;
-    for (int r = lane; r < R; r += 32) {
-        if (r >= N && !(sh.flag[r - N] & 1)) continue;
+    for (int r = tid; r < R; r += kT) {
+        if (r >= N && !(ts.flag[r - N] & 1)) continue;
         bad |= (MODE == kTreeGreedy) ? (rs.m[r] != rs.m[r]) : !stoch_row_ok(rs.m[r], rs.s[r]);
     }
-    if (__any_sync(kFull, bad)) err |= kStLogit;
-
+    if (bad) atomicOr(&ts.err, kStLogit);
+    __syncthreads();
+    const int err = ts.err;
     if (!err) {
-        for (int i = 1 + lane; i < N; i += 32) {
-            const int par = __ldg(pa + i), t = __ldg(tk + i);
+        for (int i = 1 + tid; i < N; i += kT) {
+            const int par = ts.par[i];
             bool ok;
             if (MODE == kTreeGreedy) {
-                ok = (t == rs.idx[par]);
+                ok = (ts.tok[i] == rs.idx[par]);
             } else {
                 const double lp =
-                    (f32_to_f64(pr->lt[i]) - static_cast<double>(rs.m[par])) * p.inv_t - log(rs.s[par]);
+                    (f32_to_f64(tp.lt[i]) - static_cast<double>(rs.m[par])) * p.inv_t - log(rs.s[par]);
                 const double lq =
-                    (f32_to_f64(pr->ld[i]) - static_cast<double>(rs.m[N + par])) * p.inv_t - log(rs.s[N + par]);
-                const double u = philox_uniform(p.seed, static_cast<uint32_t>(b),
-                                                static_cast<uint32_t>(i - 1), kPurposeAccept, p.offset);
-                ok = accept_test(lp, lq, u);
+                    (f32_to_f64(tp.ld[i]) - static_cast<double>(rs.m[N + par])) * p.inv_t - log(rs.s[N + par]);
+                ok = accept_test(lp, lq, tu.ua[i]);
             }
-            if (ok) sh.flag[i] |= 2;
+            if (ok) ts.flag[i] |= 2;
         }
+        __syncthreads();
+        int key = 0;
+        for (int i = tid; i < N; i += kT) {
+            bool acc = true;
+            for (int j = i; j != 0; j = ts.par[j]) acc &= (ts.flag[j] & 2) != 0;
+            if (acc) key = max(key, (static_cast<int>(ts.depth[i]) << 11) | (kMaxNodes - 1 - i));
+        }
+        key = warp_max(key);
+        if (lane == 0 && key) atomicMax(&ts.key, key);
+        __syncthreads();
     }
-    __syncwarp();
-
+    if (warp != 0) return;
     const int W = p.max_depth + 1;
     int32_t *out = p.out + static_cast<int64_t>(b) * W;
     int32_t *path = p.path ? p.path + static_cast<int64_t>(b) * W : nullptr;
-    ReqInfo info = empty_req();
-    if (err) {
-        for (int j = lane; j < W; j += 32) {
-            out[j] = -1;
-            if (path) path[j] = -1;
-        }
-        if (lane == 0) {
-            p.acc[b] = -1;
-            report(p.status, err);
-            store_req(p.req + b, info);
-        }
-        return;
-    }
-    // acceptance level by level: a node is accepted when its parent is and
-    // its test passed; the deepest accepted node wins, ties to the lowest index
-    if (lane == 0) sh.flag[0] |= 4;
-    __syncwarp();
-    for (int lvl = 1; lvl <= p.max_depth; ++lvl) {
-        for (int i = 1 + lane; i < N; i += 32)
-            if (sh.depth[i] == lvl && (sh.flag[__ldg(pa + i)] & 4) && (sh.flag[i] & 2)) sh.flag[i] |= 4;
-        __syncwarp();
-    }
-    int key = 0;  // depth << 11 | (kMaxNodes - 1 - node): larger is deeper, then lower index
-    for (int i = lane; i < N; i += 32)
-        if (sh.flag[i] & 4) key = max(key, (static_cast<int>(sh.depth[i]) << 11) | (kMaxNodes - 1 - i));
-    key = warp_max(key);
-    const int d = kMaxNodes - 1 - (key & 2047);
-    const int D = sh.depth[d];
     for (int j = lane; j < W; j += 32) {
         out[j] = -1;
         if (path) path[j] = -1;
     }
     __syncwarp();
     if (lane != 0) return;
-    for (int node = d; node != 0; node = __ldg(pa + node)) {
-        out[sh.depth[node] - 1] = __ldg(tk + node);
-        if (path) path[sh.depth[node]] = node;
+    ReqInfo info = empty_req();
+    if (err) {
+        p.acc[b] = -1;
+        report(p.status, err);
+        store_req(p.req + b, info);
+        return;
+    }
+    const int d = kMaxNodes - 1 - (ts.key & 2047);
+    const int D = ts.depth[d];
+    for (int node = d; node != 0; node = ts.par[node]) {
+        out[ts.depth[node] - 1] = ts.tok[node];
+        if (path) path[ts.depth[node]] = node;
     }
     if (path) path[0] = 0;
     p.acc[b] = D;
     if (MODE == kTreeGreedy) {
         out[D] = rs.idx[d];
-        store_req(p.req + b, info);
     } else {
         info.mode = kModeTargetRow;
         info.t_off = (static_cast<int64_t>(b) * N + d) * p.stride;
         info.mt = rs.m[d];
-        info.u = philox_uniform(p.seed, static_cast<uint32_t>(b), static_cast<uint32_t>(d),
-                                kPurposeSample, p.offset);
+        info.u = tu.us[d];
         info.out_index = b * W + D;
-        store_req(p.req + b, info);
     }
+    store_req(p.req + b, info);
 }
 
 // ------------------------------------------------------------------ pass 2
@@ -1259,10 +1293,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) k_pass1(const __grid_con
                             blockIdx.x * kWarps + warp, gridDim.x * kWarps);
 }
 
-// Decide: one block per request merges its rows (a warp per row, all rows
-// at once for up to 32) into shared memory, then warp 0 runs the decide
-// step.
-constexpr int kDecideThreads = 1024;
+// Decide: one block per request merges its rows (a warp per row) into
+// shared memory, then runs the decide step (linear: warp 0; trees: the
+// whole block, with the input-only part done before pass 1 completes).
 // partials a decide block stages in shared memory (beyond that it reads them
 // through L2): 12288 x 8 B = 96 KB
 constexpr int kDecideStageMax = 12288;
@@ -1273,6 +1306,7 @@ __global__ void __launch_bounds__(kDecideThreads) k_decide(const __grid_constant
     extern __shared__ double rowmem[];
     __shared__ TreeScratch ts;
     __shared__ TreeProbe tp;
+    __shared__ TreeUniforms tu;
     const int warp = threadIdx.x >> 5;
     RowStats rs;
     rs.s = rowmem;
@@ -1282,41 +1316,14 @@ __global__ void __launch_bounds__(kDecideThreads) k_decide(const __grid_constant
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
     DraftProbe pr;
     if (MODE == kLinear && warp == 0) pr = probe_drafts<Tag>(p, blockIdx.x);
-    // stochastic trees: the logits each node test reads are inputs, fetched
-    // before pass 1 completes (a thread per node)
-    auto fetch_tests = [&](int b) {
-        if (MODE != kTreeStochastic || b >= p.B) return;
-        const int32_t *pa = p.parents + static_cast<int64_t>(b) * p.N;
-        const int32_t *tk = p.tokens + static_cast<int64_t>(b) * p.N;
-        for (int i = 1 + threadIdx.x; i < p.N; i += kDecideThreads) {
-            const int par = __ldg(pa + i), t = __ldg(tk + i);
-            float lt = 0.f, ld = 0.f;
-            if (par >= 0 && par < i && t >= 0 && t < p.V) {
-                const int64_t off = (static_cast<int64_t>(b) * p.N + par) * p.stride + t;
-                lt = load_logit<Tag>(p.tl, off);
-                ld = load_logit<Tag>(p.dl, off);
-            }
-            tp.lt[i] = lt;
-            tp.ld[i] = ld;
-        }
-    };
-    fetch_tests(blockIdx.x);
+    // trees: everything that reads only inputs, before pass 1 completes
+    if (MODE != kLinear && static_cast<int>(blockIdx.x) < p.B) tree_prepare<Tag, MODE>(p, blockIdx.x, ts, tp, tu);
     asm volatile("griddepcontrol.wait;\n" ::: "memory");
     for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
-        if (MODE != kLinear) {
-            // draft row of node i is read iff node i has a child
-            const int32_t *pa = p.parents + static_cast<int64_t>(b) * p.N;
-            for (int i = threadIdx.x; i < p.N; i += kDecideThreads) ts.flag[i] = 0;
-            __syncthreads();
-            for (int i = 1 + threadIdx.x; i < p.N; i += kDecideThreads) {
-                const int par = __ldg(pa + i);
-                if (par >= 0 && par < i) ts.flag[par] = 1;  // every writer stores 1
-            }
-            __syncthreads();
-        }
         // the request's partials, staged in shared memory by every thread at
         // once (one round of independent loads) when they fit, then merged
-        // a warp per row
+        // a warp per row (the draft rows of nodes without children are not
+        // read)
         float2 *stg = stage_parts ? reinterpret_cast<float2 *>(rs.idx + p.R) : nullptr;
         if (stage_parts) {
             const float2 *src = p.rowpart + static_cast<int64_t>(b) * p.R * p.S;
@@ -1325,23 +1332,21 @@ __global__ void __launch_bounds__(kDecideThreads) k_decide(const __grid_constant
             __syncthreads();
         }
         for (int r = warp; r < p.R; r += kDW) {
-            if (MODE != kLinear && r >= p.N && !ts.flag[r - p.N]) continue;
+            if (MODE != kLinear && r >= p.N && !(ts.flag[r - p.N] & 1)) continue;
             merge_row<MODE>(p, b, r, rs, stg);
         }
         __syncthreads();
-        if (warp == 0) {
-            if constexpr (MODE == kLinear) {
+        if constexpr (MODE == kLinear) {
+            if (warp == 0) {
                 decide_linear<Tag>(p, b, rs, pr);
                 pr = probe_drafts<Tag>(p, b + gridDim.x);
-            } else {
-                decide_tree<Tag, MODE>(p, b, rs, ts, &tp);
             }
+        } else {
+            tree_decide<Tag, MODE>(p, b, rs, ts, tp, tu);
         }
         __syncthreads();
-        if (b + static_cast<int>(gridDim.x) < p.B) {
-            fetch_tests(b + gridDim.x);
-            __syncthreads();
-        }
+        if (MODE != kLinear && b + static_cast<int>(gridDim.x) < p.B)
+            tree_prepare<Tag, MODE>(p, b + gridDim.x, ts, tp, tu);
     }
 }
 
