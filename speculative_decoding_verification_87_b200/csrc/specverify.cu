@@ -206,19 +206,35 @@ int sm_count(int dev)
 // (the kernel itself waits for it with griddepcontrol.wait).
 template <class Kernel>
 int launch_dependent(Kernel kernel, int64_t blocks, size_t dyn, cudaStream_t st, const Params &p,
-                     int threads = kThreads)
+                     int threads = kThreads, int cluster = 1)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(blocks));
     cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = dyn;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (cluster > 1) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = static_cast<unsigned>(cluster);
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
+    }
     return cudaLaunchKernelEx(&cfg, kernel, p) == cudaSuccess ? SPEC_OK : SPEC_ECUDA;
+}
+
+// Blocks per request of the tree decide step (a cluster): enough that the
+// batch's clusters cover about two waves of SMs, at most kDecideClusterMax.
+constexpr int kDecideClusterMax = 4;
+int decide_cluster(int B, int R, int sms)
+{
+    int g = std::max(1, std::min(kDecideClusterMax, (2 * sms) / std::max(1, B)));
+    return std::min(g, R);
 }
 
 // Pass 1's static share (whole rounds of the grid's warps for about 88% of
@@ -273,8 +289,12 @@ int launch_verify(Params &p, const Layout &L, void *ws, int dtype_index, cudaStr
     if (prep_pass1(p, blocks1, st) != SPEC_OK) return SPEC_ECUDA;
     k_pass1<Tag, MODE, kMin1><<<static_cast<unsigned>(blocks1), kThreads, kRingBytes, st>>>(p);
     if (cudaGetLastError() != cudaSuccess) return SPEC_ECUDA;
-    const int64_t blocksd = std::max<int64_t>(1, std::min<int64_t>(static_cast<int64_t>(2) * sms, p.B));
-    if (launch_dependent(k_decide<Tag, MODE>, blocksd, decide_smem(p.R, p.S), st, p, kDecideThreads) != SPEC_OK)
+    const int G = MODE == kLinear ? 1 : decide_cluster(p.B, p.R, sms);
+    const int64_t blocksd =
+        G > 1 ? static_cast<int64_t>(p.B) * G
+              : std::max<int64_t>(1, std::min<int64_t>(static_cast<int64_t>(2) * sms, p.B));
+    if (launch_dependent(k_decide<Tag, MODE>, blocksd, decide_smem(p.R, p.S), st, p, kDecideThreads, G) !=
+        SPEC_OK)
         return SPEC_ECUDA;
     if (p.nP == 0) return SPEC_OK;
 

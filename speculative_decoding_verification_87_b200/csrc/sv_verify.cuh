@@ -31,6 +31,8 @@
 // waits (own asynchronous copies, the grid dependency).
 #pragma once
 
+#include <cooperative_groups.h>
+
 #include "sv_common.cuh"
 #include "sv_exp64.cuh"
 #include "sv_philox.cuh"
@@ -481,11 +483,12 @@ struct RowStats {
 // rows: (max, lowest argmax).  One warp; fixed order, so deterministic.
 template <int MODE>
 __device__ __forceinline__ void merge_row(const Params &p, int b, int r, RowStats rs,
-                                          const float2 *staged = nullptr)
+                                          const float2 *staged = nullptr, int rbase = 0)
 {
     const int lane = threadIdx.x & 31;
     // the row's partials: in global memory, or staged in shared memory
-    const float2 *part = staged ? staged + static_cast<int64_t>(r) * p.S
+    // (rows from rbase on)
+    const float2 *part = staged ? staged + static_cast<int64_t>(r - rbase) * p.S
                                 : p.rowpart + (static_cast<int64_t>(b) * p.R + r) * p.S;
     if (MODE == kTreeGreedy) {
         float bv = -INFINITY;
@@ -1302,51 +1305,68 @@ constexpr int kDecideStageMax = 12288;
 template <class Tag, int MODE>
 __global__ void __launch_bounds__(kDecideThreads) k_decide(const __grid_constant__ Params p)
 {
+    namespace cg = cooperative_groups;
     constexpr int kDW = kDecideThreads / 32;
     extern __shared__ double rowmem[];
     __shared__ TreeScratch ts;
     __shared__ TreeProbe tp;
     __shared__ TreeUniforms tu;
+    // a request is decided by a cluster of G blocks (G = 1 without a
+    // cluster launch): block `rank` merges rows [r0, r1) into the row
+    // statistics of the cluster's rank-0 block (distributed shared memory),
+    // which then runs the decide step
+    cg::cluster_group cluster = cg::this_cluster();
+    const int G = static_cast<int>(cluster.num_blocks());
+    const int rank = static_cast<int>(cluster.block_rank());
+    const int cid = blockIdx.x / G, ncl = gridDim.x / G;
+    const int RG = (p.R + G - 1) / G;
+    const int r0 = min(p.R, rank * RG), r1 = min(p.R, r0 + RG);
     const int warp = threadIdx.x >> 5;
-    RowStats rs;
+    RowStats rs;  // this block's row statistics (rank 0: the request's)
     rs.s = rowmem;
     rs.m = reinterpret_cast<float *>(rowmem + p.R);
     rs.idx = reinterpret_cast<int *>(rs.m + p.R);
-    const bool stage_parts = p.R * p.S <= kDecideStageMax;
+    RowStats rs0;  // rank 0's
+    rs0.s = cluster.map_shared_rank(rs.s, 0);
+    rs0.m = cluster.map_shared_rank(rs.m, 0);
+    rs0.idx = cluster.map_shared_rank(rs.idx, 0);
+    const bool stage_parts = (r1 - r0) * p.S <= kDecideStageMax;
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
     DraftProbe pr;
-    if (MODE == kLinear && warp == 0) pr = probe_drafts<Tag>(p, blockIdx.x);
+    if (MODE == kLinear && warp == 0) pr = probe_drafts<Tag>(p, cid);
     // trees: everything that reads only inputs, before pass 1 completes
-    if (MODE != kLinear && static_cast<int>(blockIdx.x) < p.B) tree_prepare<Tag, MODE>(p, blockIdx.x, ts, tp, tu);
+    if (MODE != kLinear && cid < p.B) tree_prepare<Tag, MODE>(p, cid, ts, tp, tu);
     asm volatile("griddepcontrol.wait;\n" ::: "memory");
-    for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
-        // the request's partials, staged in shared memory by every thread at
-        // once (one round of independent loads) when they fit, then merged
-        // a warp per row (the draft rows of nodes without children are not
-        // read)
+    for (int b = cid; b < p.B; b += ncl) {
+        // the block's rows' partials, staged in shared memory by every
+        // thread at once (one round of independent loads) when they fit,
+        // then merged a warp per row (the draft rows of nodes without
+        // children are not read)
         float2 *stg = stage_parts ? reinterpret_cast<float2 *>(rs.idx + p.R) : nullptr;
         if (stage_parts) {
-            const float2 *src = p.rowpart + static_cast<int64_t>(b) * p.R * p.S;
-            const int n = p.R * p.S;
+            const float2 *src = p.rowpart + (static_cast<int64_t>(b) * p.R + r0) * p.S;
+            const int n = (r1 - r0) * p.S;
             for (int i = threadIdx.x; i < n; i += kDecideThreads) stg[i] = __ldcg(src + i);
             __syncthreads();
         }
-        for (int r = warp; r < p.R; r += kDW) {
+        for (int r = r0 + warp; r < r1; r += kDW) {
             if (MODE != kLinear && r >= p.N && !(ts.flag[r - p.N] & 1)) continue;
-            merge_row<MODE>(p, b, r, rs, stg);
+            merge_row<MODE>(p, b, r, rs0, stg, r0);
         }
-        __syncthreads();
-        if constexpr (MODE == kLinear) {
-            if (warp == 0) {
-                decide_linear<Tag>(p, b, rs, pr);
-                pr = probe_drafts<Tag>(p, b + gridDim.x);
+        cluster.sync();  // every row's statistics are in rank 0
+        if (rank == 0) {
+            if constexpr (MODE == kLinear) {
+                if (warp == 0) {
+                    decide_linear<Tag>(p, b, rs, pr);
+                    pr = probe_drafts<Tag>(p, b + ncl);
+                }
+            } else {
+                tree_decide<Tag, MODE>(p, b, rs, ts, tp, tu);
             }
-        } else {
-            tree_decide<Tag, MODE>(p, b, rs, ts, tp, tu);
         }
         __syncthreads();
-        if (MODE != kLinear && b + static_cast<int>(gridDim.x) < p.B)
-            tree_prepare<Tag, MODE>(p, b + gridDim.x, ts, tp, tu);
+        if (MODE != kLinear && b + ncl < p.B) tree_prepare<Tag, MODE>(p, b + ncl, ts, tp, tu);
+        cluster.sync();  // rank 0 is done with the statistics before they are rewritten
     }
 }
 
