@@ -49,6 +49,32 @@ __device__ __forceinline__ float ex2_approx(float x)
     return y;
 }
 
+// Two fp32 lanes in one 64-bit register pair, and the packed fp32x2 FMA and
+// add of sm_100 (each lane rounded as its scalar instruction would be).
+__device__ __forceinline__ unsigned long long f2_pack(float lo, float hi)
+{
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(unsigned long long v, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
+                                                     unsigned long long c)
+{
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b)
+{
+    unsigned long long d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 // 2^x for x <= 0 on the FMA pipe: round x to the nearest integer n with the
 // 1.5 * 2^23 shift, evaluate 2^f (f = x - n in [-1/2, 1/2]) by its Taylor
 // polynomial of degree 6 (sum (f ln 2)^k / k!, truncation below 1.2e-7

@@ -367,14 +367,24 @@ __device__ __forceinline__ void reduce_item1(const Params &p, unsigned item, int
         const float m = lane_max<Tag>(raw);
         const float mc = (m == -INFINITY) ? 0.f : m * c;  // all -inf: every term is 0
         const float nmc = -mc;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        // entries in pairs through the packed fp32x2 FMA and add: entry e
+        // goes to sum e & 3 in index order, as four scalar sums would
+        const unsigned long long c2 = f2_pack(c, c), n2 = f2_pack(nmc, nmc);
+        unsigned long long acc2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
         for (int v = 0; v < kV; ++v) {
             float x[kVec];
             unpack<Tag>(raw[v], x);
 #pragma unroll
-            for (int e = 0; e < kVec; ++e) acc[e & 3] += ex2_approx(fmaf(x[e], c, nmc));
+            for (int e = 0; e < kVec; e += 2) {
+                float z0, z1;
+                f2_unpack(f2_fma(f2_pack(x[e], x[e + 1]), c2, n2), z0, z1);
+                acc2[(e >> 1) & 1] = f2_add(acc2[(e >> 1) & 1], f2_pack(ex2_approx(z0), ex2_approx(z1)));
+            }
         }
+        float acc[4];
+        f2_unpack(acc2[0], acc[0], acc[1]);
+        f2_unpack(acc2[1], acc[2], acc[3]);
         const float lsum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
         const float M = warp_max_nan(m);
         float sr = 0.f;
