@@ -296,3 +296,33 @@ def test_expired_waits_end_the_kernel_with_a_status(sv, orc):
     assert g["status"] == 0
     tally.add(compare_linear(g, o, w.k))
     tally.check()
+
+
+def test_both_linear_paths_agree_across_the_batch_boundary(sv, orc):
+    """Batches of one or two requests take the four-kernel path, larger ones
+    the one-kernel path.  The uniforms are keyed by request index, so the
+    first requests of a batch of 3 (one kernel), 2 and 1 (four kernels) must
+    give the same outputs (the two paths merge the normalisers in different
+    orders, so only trials inside the oracle's margins may differ), and
+    match the oracle under the parity rules."""
+    import dataclasses
+    w3 = wl.peaked_linear(seed=71, batch=3, k=6, vocab=30011, temperature=0.8, sigma=(0.5, 2.0))
+    tally = FlagTally()
+    outs = {}
+    for B in (3, 2, 1):
+        w = dataclasses.replace(w3, target=w3.target[:B].copy(), draft=w3.draft[:B].copy(),
+                                tokens=w3.tokens[:B].copy())
+        for off in range(40):
+            g = run_linear_gpu(sv, w, seed=5, offset=off)
+            o = orc.verify_linear(w.target, w.draft, w.tokens, w.vocab, w.temperature, 5, off)
+            assert g["status"] == 0
+            tally.add(compare_linear(g, o, w.k))
+            flagged = (o["smp_margin"] < 1e-5) | (o["acc_margin"] < 1e-5).any(axis=1)
+            outs[(B, off)] = (g["out"], g["acc"], flagged)
+    tally.check()
+    for off in range(40):
+        o3, a3, f3 = outs[(3, off)]
+        for B in (2, 1):
+            oB, aB, fB = outs[(B, off)]
+            same = np.all(oB == o3[:B], axis=1) & (aB == a3[:B])
+            assert np.all(same | fB | f3[:B]), (B, off)
