@@ -256,7 +256,6 @@ int launch_verify(Params &p, const Layout &L, void *ws, int dtype_index, cudaStr
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SPEC_ECUDA;
     constexpr int kMin1 = pass1_min_blocks<Tag, MODE>();
-    const size_t dyn3 = finalize_smem(p.S2);
     int per_sm1, per_sm2 = 1, sms;
     {
         std::lock_guard<std::mutex> lock(g_mu);
@@ -302,8 +301,13 @@ int launch_verify(Params &p, const Layout &L, void *ws, int dtype_index, cudaStr
         std::max<int64_t>(1, std::min<int64_t>(static_cast<int64_t>(per_sm2) * sms, ceil_div(p.nP, kWarps)));
     if (launch_dependent(k_pass2<Tag, MODE>, blocks2, StageShape<Tag>::kBytes, st, p) != SPEC_OK)
         return SPEC_ECUDA;
-    const int64_t blocks3 = std::max<int64_t>(1, std::min<int64_t>(sms, ceil_div(p.B, kWarps)));
-    return launch_dependent(k_finalize<Tag, MODE>, blocks3, dyn3, st, p);
+    // finalize: a latency chain per request, so one warp per block (one per
+    // SM while the batch fits the SMs), up to 8 warps per block beyond
+    const int fw = static_cast<int>(std::min<int64_t>(kWarps, std::max<int64_t>(1, ceil_div(p.B, sms))));
+    const int64_t blocks3 = std::max<int64_t>(1, ceil_div(p.B, fw));
+    return launch_dependent(k_finalize<Tag, MODE>, std::min<int64_t>(blocks3, static_cast<int64_t>(sms) * 8),
+                            static_cast<size_t>(fw) * 2 * sizeof(double) * (p.S2 <= kMaxS2Shared ? p.S2 : 0), st, p,
+                            32 * fw);
 }
 
 // The one-kernel linear path: clear the counters and partials, then one

@@ -1453,12 +1453,12 @@ __global__ void __launch_bounds__(kThreads) k_finalize(const __grid_constant__ P
 {
     extern __shared__ double wdyn[];
     __shared__ double tab[kExp2Tab];
-    const int warp = threadIdx.x >> 5;
-    for (int j = threadIdx.x; j < kExp2Tab; j += kThreads) tab[j] = p.exp2tab[j];
+    const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    for (int j = threadIdx.x; j < kExp2Tab; j += blockDim.x) tab[j] = p.exp2tab[j];
     __syncthreads();
     const bool w_shared = p.S2 <= kMaxS2Shared;
     asm volatile("griddepcontrol.wait;\n" ::: "memory");
-    for (int b = blockIdx.x * kWarps + warp; b < p.B; b += gridDim.x * kWarps) {
+    for (int b = blockIdx.x * nw + warp; b < p.B; b += gridDim.x * nw) {
         if (__ldcg(&p.req[b].mode) == kModeNone) continue;
         double *W = w_shared ? wdyn + 2 * warp * p.S2 : p.p2w + 2 * static_cast<int64_t>(b) * p.S2;
         finalize<Tag>(p, b, tab, W, W + p.S2);
