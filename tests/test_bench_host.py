@@ -78,3 +78,34 @@ def test_empirical_alpha():
 def test_whole_job_rates():
     # 64 requests a step, 10 steps, 2 ranks, 5 ms: requests and rows per second
     assert bench.whole_job_rate(64, 10, 2, 5.0) == 64 * 10 * 2 / 0.005
+
+
+def test_greedy_forms_share_the_workload_bytes():
+    # the streamed and the workspace-free greedy forms time the same call on
+    # the same rows: identical row and byte counts, distinct workload names
+    w = wl.greedy_linear(seed=3, batch=8, k=4, vocab=1000)
+    rows, full, cfg = bench.workload_facts("greedy", w)
+    rows_c, full_c, cfg_c = bench.workload_facts("greedy-cluster", w)
+    assert (rows, full) == (rows_c, full_c)
+    assert cfg["workload"] != cfg_c["workload"] and "workspace-free" in cfg_c["workload"]
+    assert "greedy-cluster" in bench.KERNEL_OF
+
+
+def test_traffic_records_are_keyed_and_current():
+    # every committed record names a workload the bench produces, a summary
+    # that exists, and carries DRAM bytes; a record whose sources changed
+    # since its capture reads as unmeasured
+    import json
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        rec = json.load(f)
+    assert rec
+    for key, e in rec.items():
+        assert os.path.exists(os.path.join(ROOT, e["summary"])), key
+        assert e["dram_read_bytes"] > 0 and e["dram_write_bytes"] >= 0
+        assert e["tu"] in ("specverify.cu", "walk.cu")
+        traffic, src = bench.measured_traffic(key)
+        if e["tu_sha256"] == bench.tu_digest(e["tu"]):
+            assert traffic == e["dram_read_bytes"] + e["dram_write_bytes"] and src == e["summary"]
+        else:
+            assert traffic is None
+    assert bench.measured_traffic("no such workload") == (None, None)
