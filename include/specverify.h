@@ -102,12 +102,13 @@ enum {
 
 /*
  * Bytes of device workspace a call needs for `batch` requests with
- * `rows_per_req` logit rows each (linear: 2k+1; tree: 2*num_nodes) over a
- * vocabulary of `vocab` entries.  The workspace holds per-row partial
- * normalisers, per-request decisions and per-request completion counters.
- * It must be 256-byte aligned; it needs no initialisation (each call's
- * kernels first clear what they count with) and its contents are undefined
- * between calls.  Two calls that may run concurrently need two workspaces.
+ * `rows_per_req` logit rows each (linear: 2k+1; greedy with a workspace:
+ * k+1; tree: 2*num_nodes) over a vocabulary of `vocab` entries.  The
+ * workspace holds per-row partial normalisers (or partial argmaxes),
+ * per-request decisions, counters and the draw's partial sums.  It must be
+ * 256-byte aligned; it needs no initialisation (each call first clears, on
+ * its stream, what it counts with) and its contents are undefined between
+ * calls.  Two calls that may run concurrently need two workspaces.
  * Returns 0 for invalid arguments.
  */
 SPECVERIFY_API size_t spec_verify_workspace_size(int batch, int rows_per_req, int vocab);
